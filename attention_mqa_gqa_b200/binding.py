@@ -1,0 +1,166 @@
+"""ctypes binding of ``libattn_b200.so`` (declared in ``include/attn_b200.h``).
+
+Argument marshalling only: every step of the attention runs in the CUDA
+library.  Torch tensors supply device pointers, strides and the stream; the
+library must be built (``python -m attention_mqa_gqa_b200.build``) and a
+missing library is an error, never a fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_EWORKSPACE, ATTN_ECUDA, ATTN_ETIMEOUT = range(6)
+ATTN_BF16, ATTN_FP16 = 0, 1
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("h", ctypes.c_int64), ("s", ctypes.c_int64)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
+                ("head_blocks", ctypes.c_int), ("num_splits", ctypes.c_int),
+                ("split_tokens", ctypes.c_int), ("dv_parts", ctypes.c_int),
+                ("grid_ctas", ctypes.c_int64), ("workspace_bytes", ctypes.c_size_t)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} ({status})" if what else status_str(status))
+
+
+# Every symbol include/attn_b200.h declares (checked by the CPU test suite).
+EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_last_device_error",
+           "attn_status_str", "attn_version")
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing "
+                           "(run python -m attention_mqa_gqa_b200.build)")
+    lib = ctypes.CDLL(path)
+    i32, i64, sz, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+    lib.attn_plan.restype = i32
+    lib.attn_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(Plan)]
+    lib.attn_workspace_bytes.restype = sz
+    lib.attn_workspace_bytes.argtypes = [i32] * 7
+    lib.attn_fwd.restype = i32
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
+                             ctypes.c_float, i32, i32, Strides, Strides, Strides, Strides,
+                             vp, sz, vp]
+    lib.attn_last_device_error.restype = i32
+    lib.attn_last_device_error.argtypes = [vp]
+    lib.attn_status_str.restype = ctypes.c_char_p
+    lib.attn_status_str.argtypes = [i32]
+    lib.attn_version.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return load().attn_status_str(int(status)).decode()
+
+
+def version() -> str:
+    return load().attn_version().decode()
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return ATTN_BF16
+    if dt == torch.float16:
+        return ATTN_FP16
+    raise TypeError(f"unsupported element type {dt}")
+
+
+def plan(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype=torch.bfloat16, num_sms: int = 0) -> dict:
+    pl = Plan()
+    code = dtype_code(dtype) if isinstance(dtype, torch.dtype) else int(dtype)
+    rc = load().attn_plan(B, Hq, Hkv, Sq, max_skv, d_k, d_v, code, num_sms, ctypes.byref(pl))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_plan")
+    return pl.as_dict()
+
+
+def workspace_bytes(B, Hq, Hkv, Sq, max_skv, d_k, d_v) -> int:
+    return int(load().attn_workspace_bytes(B, Hq, Hkv, Sq, max_skv, d_k, d_v))
+
+
+def _strides4(t: torch.Tensor) -> Strides:
+    if t.dim() != 4 or t.stride(-1) != 1:
+        raise ValueError("expected a [B, H, S, d] tensor with a contiguous last dimension")
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def fwd_raw(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v, scale, causal,
+            dtype_code_, sq: Strides, sk: Strides, sv: Strides, so: Strides,
+            workspace_ptr, workspace_nbytes, stream_ptr) -> int:
+    """Direct call with raw pointers (ints); returns the status code."""
+    return load().attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v,
+                           float(scale), int(causal), dtype_code_, sq, sk, sv, so,
+                           workspace_ptr, workspace_nbytes, stream_ptr)
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+             skv: torch.Tensor, max_skv: int, scale: float, causal: bool = True,
+             lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+             stream: torch.cuda.Stream | None = None) -> None:
+    """Enqueue the forward on ``stream`` (default: torch's current stream).
+
+    q [B,Hq,Sq,d_k], k [B,Hkv,S,d_k], v [B,Hkv,S,d_v], out [B,Hq,Sq,d_v]
+    (device tensors, last dim contiguous, any 16-byte-aligned strides);
+    skv int32 [B] device; lse fp32 [B,Hq,Sq] contiguous or None; workspace a
+    device byte tensor of at least ``workspace_bytes(...)`` bytes."""
+    B, Hq, Sq, d_k = q.shape
+    Hkv, d_v = k.shape[1], v.shape[-1]
+    if skv.dtype != torch.int32:
+        raise TypeError("skv must be int32")
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise TypeError("lse must be a contiguous float32 tensor")
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                 lse.data_ptr() if lse is not None else None,
+                 B, Hq, Hkv, Sq, skv.data_ptr(), int(max_skv), d_k, d_v, scale, causal,
+                 dtype_code(q.dtype), _strides4(q), _strides4(k), _strides4(v), _strides4(out),
+                 ws_ptr, ws_n, st.cuda_stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+
+
+def last_device_error(stream: torch.cuda.Stream | None = None) -> int:
+    st = stream if stream is not None else torch.cuda.current_stream()
+    return int(load().attn_last_device_error(st.cuda_stream))
+
+
+def attention(q, k, v, skv, max_skv, scale, causal=True, with_lse=True, workspace=None,
+              stream=None):
+    """Allocate out (and lse, workspace) with torch and run :func:`attn_fwd`."""
+    B, Hq, Sq, _ = q.shape
+    d_v = v.shape[-1]
+    out = torch.empty(B, Hq, Sq, d_v, dtype=q.dtype, device=q.device)
+    lse = torch.empty(B, Hq, Sq, dtype=torch.float32, device=q.device) if with_lse else None
+    if workspace is None:
+        n = workspace_bytes(B, Hq, k.shape[1], Sq, int(max_skv), q.shape[-1], d_v)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    attn_fwd(q, k, v, out, skv, max_skv, scale, causal, lse, workspace, stream)
+    return out, lse

@@ -1,0 +1,306 @@
+// attn_api.cu -- the C ABI declared in include/attn_b200.h: argument
+// validation, the launch plan (prefill vs split-KV decode, split sizes),
+// TMA tensor maps, and kernel launches on the caller's stream.
+//
+// Single translation unit: the kernels (and the device error word they
+// share) are compiled here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn_b200.h"
+#include "decode_kernel.cuh"
+#include "prefill_kernel.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+constexpr int kDecodeTile = 128;
+
+// ------------------------------------------------------------------ driver
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, H, S, D] tensor (innermost D), box = 64 columns x 128
+// rows, 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t S,
+              uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  // strides of extent-1 dimensions are irrelevant; give them valid values
+  if (S == 1) ss = (int64_t)D;
+  if (H == 1) sh = ss * (int64_t)S;
+  if (B == 1) sb = sh * (int64_t)H;
+  cuuint64_t dims[4] = {D, S, H, B};
+  cuuint64_t strides[3] = {(cuuint64_t)ss * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool strides_ok(const attn_strides_t& s) {
+  return s.b >= 0 && s.h >= 0 && s.s >= 0 && s.b % 8 == 0 && s.h % 8 == 0 && s.s % 8 == 0;
+}
+
+bool shape_supported(int Sq, int d_k, int d_v) {
+  if (Sq > 1) return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512);
+  return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512) || (d_k == 576 && d_v == 512);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v,
+                        attn_dtype_t dtype, int num_sms, attn_plan_t* pl) {
+  if (!pl) return ATTN_EINVAL;
+  std::memset(pl, 0, sizeof(*pl));
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || max_skv <= 0 || d_k <= 0 || d_v <= 0)
+    return ATTN_EINVAL;
+  if (Hq % Hkv != 0) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_EINVAL;
+  if (!shape_supported(Sq, d_k, d_v)) return ATTN_EUNSUPPORTED;
+  if (num_sms <= 0) num_sms = device_sm_count();
+  const int G = Hq / Hkv;
+  if (Sq > 1) {
+    pl->path = 0;
+    pl->dv_parts = d_v / (d_v >= 512 ? 256 : 128);
+    const int64_t n_qt = (Sq + 127) / 128;
+    pl->grid_ctas = n_qt * Hq * (int64_t)B * pl->dv_parts;
+    if (pl->grid_ctas > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
+    pl->workspace_bytes = 0;
+    return ATTN_OK;
+  }
+  pl->path = 1;
+  const int NH = d_k == 576 ? 64 : 16;
+  pl->heads_per_cta = NH;
+  pl->head_blocks = (G + NH - 1) / NH;
+  const int64_t units = (int64_t)B * Hkv * pl->head_blocks;
+  const int tiles = (max_skv + kDecodeTile - 1) / kDecodeTile;
+  const int ctas_per_sm = d_k == 576 ? 1 : 2;
+  // Aim for about three resident waves of CTAs so the ragged per-sequence
+  // lengths (unknown to the host) even out across the SMs.
+  const int64_t target = (int64_t)num_sms * ctas_per_sm * 3;
+  int64_t want = (target + units - 1) / units;
+  if (want < 1) want = 1;
+  int split_tiles = (int)((tiles + want - 1) / want);
+  if (split_tiles < 1) split_tiles = 1;
+  pl->split_tokens = split_tiles * kDecodeTile;
+  pl->num_splits = (tiles + split_tiles - 1) / split_tiles;
+  pl->grid_ctas = units * pl->num_splits;
+  if (B > 65535 || Hkv > 65535 || (int64_t)pl->head_blocks * pl->num_splits > 0x7fffffffLL)
+    return ATTN_EUNSUPPORTED;
+  const size_t n = (size_t)B * Hq * pl->num_splits;
+  pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float));
+  return ATTN_OK;
+}
+
+template <typename K>
+void set_smem(K kernel, int bytes) {
+  // idempotent; cheap enough to repeat per launch
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int DK, int DV, int NH, bool BF16>
+attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
+                            const attn::DecodeParams& dp, const attn::CombineParams& cp,
+                            const attn_plan_t& pl, cudaStream_t st) {
+  using Tr = attn::DecodeTraits<DK, DV, NH>;
+  auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
+  set_smem(kern, Tr::SMEM_BYTES);
+  dim3 grid(pl.head_blocks * pl.num_splits, dp.B, dp.Hkv);
+  kern<<<grid, 192, Tr::SMEM_BYTES, st>>>(mk, mv, dp);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  return ATTN_OK;
+}
+
+template <int DK, int DVH, bool BF16>
+attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                             const attn::PrefillParams& pp, const attn_plan_t& pl,
+                             cudaStream_t st) {
+  using Tr = attn::PrefillTraits<DK, DVH>;
+  auto kern = attn::prefill_kernel<DK, DVH, BF16>;
+  set_smem(kern, Tr::SMEM_BYTES);
+  kern<<<(unsigned)pl.grid_ctas, 192, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_plan(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v,
+                        attn_dtype_t dtype, int num_sms, attn_plan_t* plan) {
+  return plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype, num_sms, plan);
+}
+
+size_t attn_workspace_bytes(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v) {
+  attn_plan_t pl;
+  if (plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, ATTN_BF16, 0, &pl) != ATTN_OK) return 0;
+  return pl.workspace_bytes;
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Sq, const int32_t* skv_per_seq, int max_skv,
+                       int d_k, int d_v, float scale, int causal, attn_dtype_t dtype,
+                       attn_strides_t sq, attn_strides_t sk, attn_strides_t sv,
+                       attn_strides_t so, void* workspace, size_t workspace_bytes,
+                       void* cuda_stream) {
+  // ---- validation (nothing touches the GPU before this passes)
+  if (!q || !k || !v || !out || !skv_per_seq) return ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_EINVAL;
+  if (reinterpret_cast<uintptr_t>(skv_per_seq) & 3u) return ATTN_EINVAL;
+  if (!strides_ok(sq) || !strides_ok(sk) || !strides_ok(sv) || !strides_ok(so)) return ATTN_EINVAL;
+  if (causal != 0 && causal != 1) return ATTN_EINVAL;
+  if (!std::isfinite(scale)) return ATTN_EINVAL;
+  attn_plan_t pl;
+  attn_status_t rc = plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype, 0, &pl);
+  if (rc != ATTN_OK) return rc;
+  if ((Sq > 1 && sq.s == 0) || sk.s == 0 || sv.s == 0 || (Sq > 1 && so.s == 0)) return ATTN_EINVAL;
+  if (pl.workspace_bytes > 0) {
+    if (!workspace || !aligned16(workspace)) return ATTN_EWORKSPACE;
+    if (workspace_bytes < pl.workspace_bytes) return ATTN_EWORKSPACE;
+  }
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  const bool bf16 = dtype == ATTN_BF16;
+  const int G = Hq / Hkv;
+
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b)) return ATTN_ECUDA;
+  if (!make_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b)) return ATTN_ECUDA;
+
+  if (pl.path == 1) {
+    attn::DecodeParams dp{};
+    dp.q = q;
+    dp.q_sb = sq.b;
+    dp.q_sh = sq.h;
+    dp.skv = skv_per_seq;
+    const size_t n = (size_t)B * Hq * pl.num_splits;
+    dp.ws_o = reinterpret_cast<float*>(workspace);
+    dp.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                         align256(n * d_v * sizeof(float)));
+    dp.B = B;
+    dp.Hq = Hq;
+    dp.Hkv = Hkv;
+    dp.G = G;
+    dp.num_splits = pl.num_splits;
+    dp.split_tiles = pl.split_tokens / kDecodeTile;
+    dp.head_blocks = pl.head_blocks;
+    dp.scale_log2 = scale_log2;
+    dp.timeout_ns = kDefaultTimeoutNs;
+    attn::CombineParams cp{};
+    cp.ws_o = dp.ws_o;
+    cp.ws_lse = dp.ws_lse;
+    cp.skv = skv_per_seq;
+    cp.out = out;
+    cp.o_sb = so.b;
+    cp.o_sh = so.h;
+    cp.lse = lse;
+    cp.B = B;
+    cp.Hq = Hq;
+    cp.DV = d_v;
+    cp.num_splits = pl.num_splits;
+    cp.split_tokens = pl.split_tokens;
+    if (d_k == 128)
+      return bf16 ? launch_decode<128, 128, 16, true>(mk, mv, dp, cp, pl, st)
+                  : launch_decode<128, 128, 16, false>(mk, mv, dp, cp, pl, st);
+    if (d_k == 512)
+      return bf16 ? launch_decode<512, 512, 16, true>(mk, mv, dp, cp, pl, st)
+                  : launch_decode<512, 512, 16, false>(mk, mv, dp, cp, pl, st);
+    return bf16 ? launch_decode<576, 512, 64, true>(mk, mv, dp, cp, pl, st)
+                : launch_decode<576, 512, 64, false>(mk, mv, dp, cp, pl, st);
+  }
+
+  CUtensorMap mq;
+  if (!make_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b)) return ATTN_ECUDA;
+  attn::PrefillParams pp{};
+  pp.out = out;
+  pp.o_sb = so.b;
+  pp.o_sh = so.h;
+  pp.o_ss = so.s;
+  pp.lse = lse;
+  pp.skv = skv_per_seq;
+  pp.B = B;
+  pp.Hq = Hq;
+  pp.Hkv = Hkv;
+  pp.G = G;
+  pp.Sq = Sq;
+  pp.n_qtiles = (Sq + 127) / 128;
+  pp.dv_parts = pl.dv_parts;
+  pp.scale_log2 = scale_log2;
+  pp.causal = causal;
+  pp.timeout_ns = kDefaultTimeoutNs;
+  if (d_k == 128)
+    return bf16 ? launch_prefill<128, 128, true>(mq, mk, mv, pp, pl, st)
+                : launch_prefill<128, 128, false>(mq, mk, mv, pp, pl, st);
+  return bf16 ? launch_prefill<512, 256, true>(mq, mk, mv, pp, pl, st)
+              : launch_prefill<512, 256, false>(mq, mk, mv, pp, pl, st);
+}
+
+attn_status_t attn_last_device_error(void* cuda_stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ECUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, attn::g_attn_error, sizeof(word)) != cudaSuccess)
+    return ATTN_ECUDA;
+  if (word != 0 && cudaMemcpyToSymbol(attn::g_attn_error, &zero, sizeof(zero)) != cudaSuccess)
+    return ATTN_ECUDA;
+  return word ? ATTN_ETIMEOUT : ATTN_OK;
+}
+
+const char* attn_status_str(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_EINVAL: return "invalid argument";
+    case ATTN_EUNSUPPORTED: return "unsupported shape or type";
+    case ATTN_EWORKSPACE: return "workspace missing or too small";
+    case ATTN_ECUDA: return "CUDA error";
+    case ATTN_ETIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* attn_version(void) { return "0.1.0"; }
+
+}  // extern "C"

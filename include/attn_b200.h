@@ -1,0 +1,141 @@
+/*
+ * attn_b200.h -- C ABI of libattn_b200.so: fused grouped-query attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * Operation ("带你了解Attention,从MHA到DeepSeek" section 1.2; "GQA和MLA详解"
+ * sections 1-3; "Full 路线：保留 softmax，压缩 K/V 表示" sections 三 and 4.3):
+ *
+ *   out[b,h,i,:] = sum_j softmax_j( scale * q[b,h,i,:] . k[b,h/G,j,:] ) v[b,h/G,j,:]
+ *   lse[b,h,i]   = ln sum_j exp( scale * q[b,h,i,:] . k[b,h/G,j,:] )
+ *
+ * with G = Hq / Hkv query heads per K/V head (G = Hq is MQA, G = 1 is MHA;
+ * query head h reads kv head h / G, as repeat_interleave does), j running
+ * over the visible keys of sequence b: j < skv[b], and with `causal` set,
+ * j <= i + skv[b] - Sq (bottom-right alignment: a single decode query sees
+ * every key).  A row with no visible key yields out = 0 and lse = -inf.
+ *
+ * Absorbed MLA decode ("Full 路线" section 4.3: W_UK folded into the query,
+ * the cache holds rows [c_kv (512) | k_pe (64)]) is the same call with
+ * d_k = 576, d_v = 512, Hkv = 1 and v pointing at the same rows as k (the
+ * first 512 columns): the kernel then loads each cached row once.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are row-major [B, H, S, d] addressed with element strides
+ *   (attn_strides_t: b, h, s); the innermost (d) stride is 1.  All device
+ *   pointers must be 16-byte aligned and every stride a multiple of 8
+ *   elements (16 bytes), which tensor-memory-access (TMA) copies require.
+ * - q: [B, Hq, Sq, d_k]; k: [B, Hkv, >= max_skv, d_k]; v: [B, Hkv,
+ *   >= max_skv, d_v]; out: [B, Hq, Sq, d_v] (same element type as q);
+ *   lse: [B, Hq, Sq] fp32, contiguous, may be NULL.
+ * - Key rows at or past skv[b] (up to max_skv) are never weighted but are
+ *   read by whole 128-row tiles; they must hold finite numbers.
+ * - Ownership: the caller owns every buffer (q, k, v, out, lse, skv,
+ *   workspace).  The library allocates no device memory and never
+ *   synchronises the stream inside attn_fwd; all work is enqueued on
+ *   `cuda_stream` (a cudaStream_t; NULL = the legacy default stream).
+ * - Errors: argument problems are reported before anything is launched;
+ *   device-side waits that exceed their time limit set a device error word
+ *   read by attn_last_device_error().
+ *
+ * Supported shapes: (d_k, d_v) in {(128,128), (512,512)} for prefill
+ * (Sq > 1) and decode (Sq == 1); (576, 512) for decode.  Element type bf16
+ * or fp16.  Anything else returns ATTN_EUNSUPPORTED; there is no fallback.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_EINVAL = 1,        /* bad pointer, size, stride or alignment            */
+  ATTN_EUNSUPPORTED = 2,  /* valid request outside the supported shapes        */
+  ATTN_EWORKSPACE = 3,    /* workspace missing or smaller than required        */
+  ATTN_ECUDA = 4,         /* a CUDA runtime/driver call or launch failed       */
+  ATTN_ETIMEOUT = 5       /* a device-side wait gave up (see attn_last_device_error) */
+} attn_status_t;
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype_t;
+
+/* Element strides of a [B, H, S, d] tensor; the d stride is always 1. */
+typedef struct {
+  int64_t b, h, s;
+} attn_strides_t;
+
+/* What attn_fwd will launch for a problem (host-side plan, no GPU needed). */
+typedef struct {
+  int path;            /* 0 = prefill kernel, 1 = split-KV decode + combine      */
+  int heads_per_cta;   /* decode: query heads packed into one CTA (MMA N)       */
+  int head_blocks;     /* decode: CTAs per (b, kv head) along the query heads   */
+  int num_splits;      /* decode: KV splits per sequence                        */
+  int split_tokens;    /* decode: keys per split (multiple of 128)              */
+  int dv_parts;        /* prefill: CTAs sharing one q tile, each owning d_v/dv_parts columns */
+  int64_t grid_ctas;   /* CTAs of the main kernel                               */
+  size_t workspace_bytes;
+} attn_plan_t;
+
+/*
+ * Plan a call.  `num_sms` <= 0 means "ask the current device" (148 if no
+ * device is visible).  Pure host computation; returns ATTN_EINVAL /
+ * ATTN_EUNSUPPORTED under the same rules as attn_fwd.
+ * Source: "GQA和MLA详解" section 1 (prefill is the quadratic T x T phase,
+ * decode reads the whole cache once per step and is bandwidth-bound).
+ */
+attn_status_t attn_plan(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v,
+                        attn_dtype_t dtype, int num_sms, attn_plan_t* plan);
+
+/*
+ * Workspace bytes attn_fwd needs for this problem on the current device
+ * (0 for prefill).  Decode stores per-split partial outputs (fp32
+ * [B, Hq, splits, d_v]) and partial LSEs (fp32 [B, Hq, splits]) there.
+ * Returns 0 for arguments attn_plan rejects.
+ */
+size_t attn_workspace_bytes(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v);
+
+/*
+ * The forward pass (definition at the top of this file).
+ *   skv_per_seq: device pointer, int32 [B], 0 <= skv[b] <= max_skv (not
+ *                checked on the device).
+ *   max_skv:     host value, the row extent of k and v (>= 1).
+ *   scale:       multiplies q.k before the softmax (1/sqrt(d_k) for plain
+ *                attention; 1/sqrt(192) for DeepSeek-V3 MLA, whose score
+ *                scale follows the un-absorbed head width).
+ *   causal:      0 or 1 (bottom-right alignment, see above).
+ *   workspace:   device buffer of at least attn_workspace_bytes(...) bytes,
+ *                16-byte aligned (may be NULL when that is 0).  Concurrent
+ *                calls must not share a workspace.
+ * Returns ATTN_OK once the kernels are enqueued.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Sq,
+                       const int32_t* skv_per_seq, int max_skv,
+                       int d_k, int d_v, float scale, int causal, attn_dtype_t dtype,
+                       attn_strides_t sq, attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * Synchronises `cuda_stream`, then reads and clears the current device's
+ * error word.  ATTN_OK if no kernel of this library reported a problem
+ * since the last call, ATTN_ETIMEOUT if a device-side wait gave up (the
+ * outputs of that launch are undefined), ATTN_ECUDA if the stream itself
+ * reports an error.
+ */
+attn_status_t attn_last_device_error(void* cuda_stream);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_str(attn_status_t status);
+
+/* Library version, e.g. "0.1.0". */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,172 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases compare every output element; the full-size workloads compare
+sampled rows (the oracle evaluates those rows one by one).  Tolerance:
+|gpu - oracle| <= 1e-2 + 1e-2*|oracle| per element, |dLSE| <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from attention_mqa_gqa_b200 import workloads as wl
+from tests.helpers import compare, oracle_full, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from attention_mqa_gqa_b200 import binding, build
+
+    build.build()
+    binding.load()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _case(B, Hq, Hkv, Sq, skv, dk, dv, dtype=torch.bfloat16, causal=True, mla=False, seed=0,
+          max_skv=None, scale=None):
+    w, inp = wl.make_case(B, Hq, Hkv, Sq, skv, dk, dv, dtype=dtype, causal=causal, mla=mla,
+                          seed=seed, max_skv=max_skv, scale=scale)
+    dev = to_device(inp)
+    out, lse = run_gpu(w, dev)
+    ref_o, ref_l = oracle_full(w, inp)
+    return compare(out, lse, ref_o, ref_l, what=w.name)
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 1), (16, 2), (4, 4), (32, 2), (40, 2)])
+def test_decode_d128(Hq, Hkv):
+    _case(3, Hq, Hkv, 1, [1, 129, 700], 128, 128, seed=Hq + Hkv)
+
+
+@pytest.mark.parametrize("skv", [[1], [127], [128], [129], [255, 256, 257], [3000, 17, 1024]])
+def test_decode_d128_ragged(skv):
+    _case(len(skv), 8, 1, 1, skv, 128, 128, seed=sum(skv))
+
+
+@pytest.mark.parametrize("Hq,skv", [(16, [1, 129, 700, 2049]), (4, [300, 5]), (16, [4097])])
+def test_decode_mqa_d512(Hq, skv):
+    _case(len(skv), Hq, 1, 1, skv, 512, 512, seed=7)
+
+
+@pytest.mark.parametrize("Hq,skv", [(128, [1, 200, 1500]), (16, [513, 64]), (64, [2000])])
+def test_decode_mla(Hq, skv):
+    _case(len(skv), Hq, 1, 1, skv, 576, 512, mla=True, seed=11, scale=1 / math.sqrt(192))
+
+
+def test_decode_fp16():
+    _case(2, 16, 1, 1, [333, 1000], 512, 512, dtype=torch.float16, seed=3)
+
+
+def test_decode_zero_length_sequence():
+    _case(3, 16, 1, 1, [0, 300, 0], 512, 512, seed=5, max_skv=300)
+
+
+def test_decode_strided_views():
+    """q/out as views with padded strides; K/V as slices of a wider buffer."""
+    from attention_mqa_gqa_b200 import binding
+    from oracle import c_oracle
+
+    g = torch.Generator().manual_seed(9)
+    B, Hq, Hkv, S, d = 2, 16, 2, 400, 128
+    qbig = torch.randn(B, Hq, 1, d + 64, generator=g).to(torch.bfloat16)
+    kbig = torch.randn(B, Hkv, S, d + 128, generator=g).to(torch.bfloat16)
+    vbig = torch.randn(B, Hkv, S, d + 64, generator=g).to(torch.bfloat16)
+    q, k, v = qbig[..., 8:8 + d], kbig[..., 64:64 + d], vbig[..., :d]
+    skv = torch.tensor([400, 211], dtype=torch.int32)
+    qd, kd, vd = qbig.cuda()[..., 8:8 + d], kbig.cuda()[..., 64:64 + d], vbig.cuda()[..., :d]
+    outbig = torch.zeros(B, Hq, 1, d + 32, dtype=torch.bfloat16, device="cuda")
+    out = outbig[..., 16:16 + d]
+    lse = torch.empty(B, Hq, 1, device="cuda")
+    ws = torch.empty(binding.workspace_bytes(B, Hq, Hkv, 1, S, d, d), dtype=torch.uint8, device="cuda")
+    binding.attn_fwd(qd, kd, vd, out, skv.cuda(), S, 0.1, True, lse, ws)
+    torch.cuda.synchronize()
+    ref_o, ref_l = c_oracle.attention_fwd(q, k, v, skv.tolist(), 0.1, True)
+    compare(out, lse, ref_o, ref_l, "strided decode")
+    assert (outbig[..., :16] == 0).all() and (outbig[..., 16 + d:] == 0).all()
+
+
+# ----------------------------------------------------------------- prefill
+
+@pytest.mark.parametrize("Sq,skv,causal", [(200, 200, True), (200, 200, False), (128, 128, True),
+                                           (257, 257, True), (130, 300, True), (1, 1, True)])
+def test_prefill_d128(Sq, skv, causal):
+    if Sq == 1:
+        pytest.skip("Sq == 1 takes the decode path")
+    _case(1, 4, 2, Sq, [skv], 128, 128, causal=causal, seed=Sq)
+
+
+def test_prefill_d128_varlen_bottom_right():
+    """Two sequences with fewer keys than queries in one: bottom-right
+    alignment leaves the first rows with no visible key (out 0, lse -inf)."""
+    _case(2, 8, 1, 150, [300, 100], 128, 128, causal=True, seed=21, max_skv=300)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_prefill_d512(dtype):
+    _case(1, 16, 1, 300, [300], 512, 512, dtype=dtype, causal=True, seed=4)
+
+
+def test_prefill_d512_noncausal_ragged():
+    _case(2, 4, 1, 129, [129, 129], 512, 512, causal=False, seed=6)
+
+
+def test_prefill_mqa_tiny_workload():
+    """The MQA d=512 fp16 prefill workload (B=1, Hq=16, S=128) in full."""
+    w = wl.WORKLOADS["mqa_prefill_tiny"]
+    inp = wl.make_inputs(w)
+    out, lse = run_gpu(w, to_device(inp))
+    ref_o, ref_l = oracle_full(w, inp)
+    compare(out, lse, ref_o, ref_l, w.name)
+
+
+# ------------------------------------------------------------- determinism
+
+def test_bitwise_reproducible():
+    w, inp = wl.make_case(4, 16, 1, 1, [5000, 100, 2000, 7000], 512, 512, seed=13)
+    dev = to_device(inp)
+    a, la = run_gpu(w, dev)
+    b, lb = run_gpu(w, dev)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+    w, inp = wl.make_case(1, 4, 1, 600, [600], 128, 128, seed=14)
+    dev = to_device(inp)
+    a, la = run_gpu(w, dev)
+    b, lb = run_gpu(w, dev)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+# ------------------------------------------------------- full-size workloads
+
+def _sampled(name, n_pairs=12, n_rows=48, seed=0):
+    from oracle import attention as npo
+    from oracle import c_oracle
+
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w)
+    out, lse = run_gpu(w, to_device(inp))
+    rng = np.random.default_rng(seed)
+    if w.is_decode:
+        pairs = [(int(rng.integers(w.B)), int(rng.integers(w.Hq))) for _ in range(n_pairs)]
+        pairs += [(0, 0), (w.B - 1, w.Hq - 1)]
+        ref_o, ref_l = c_oracle.attention_fwd(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(),
+                                              w.scale, w.causal, pairs=pairs)
+        for (b, h) in pairs:
+            compare(out[b, h], lse[b, h], ref_o[b, h], ref_l[b, h], f"{name} b={b} h={h}")
+    else:
+        rows = [(int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.Sq)))
+                for _ in range(n_rows)]
+        rows += [(0, 0, 0), (w.B - 1, w.Hq - 1, w.Sq - 1), (0, w.Hq - 1, 127), (0, 1, 128)]
+        ref_o, ref_l = npo.attention_rows(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(),
+                                          w.scale, w.causal, rows)
+        for r, (b, h, i) in enumerate(rows):
+            compare(out[b, h, i], lse[b, h, i], ref_o[r], ref_l[r], f"{name} row {(b, h, i)}")
+
+
+@pytest.mark.parametrize("name", ["mqa_decode", "gqa_decode", "mla_decode", "mqa_prefill",
+                                  "gqa_prefill"])
+def test_full_workload_sampled(name):
+    _sampled(name)

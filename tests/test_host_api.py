@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI (no GPU): the library builds and loads,
+exports every entry point the header declares, plans correctly, and rejects
+bad arguments before anything reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_mqa_gqa_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(binding.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert binding.status_str(code) and binding.status_str(code) != "unknown status"
+    assert binding.version().count(".") == 2
+
+
+def test_plan_decode_invariants(lib):
+    for (B, Hq, Hkv, S, dk, dv) in [(32, 16, 1, 8192, 512, 512), (64, 64, 8, 4096, 128, 128),
+                                    (64, 128, 1, 16384, 576, 512), (1, 8, 8, 1, 128, 128),
+                                    (3, 40, 2, 1000, 128, 128)]:
+        pl = binding.plan(B, Hq, Hkv, 1, S, dk, dv, num_sms=148)
+        G = Hq // Hkv
+        assert pl["path"] == 1
+        assert pl["heads_per_cta"] == (64 if dk == 576 else 16)
+        assert pl["head_blocks"] == -(-G // pl["heads_per_cta"])
+        assert pl["split_tokens"] % 128 == 0
+        assert pl["num_splits"] * pl["split_tokens"] >= S > (pl["num_splits"] - 1) * pl["split_tokens"]
+        assert pl["grid_ctas"] == B * Hkv * pl["head_blocks"] * pl["num_splits"]
+        n = B * Hq * pl["num_splits"]
+        r256 = lambda x: (x + 255) // 256 * 256
+        assert pl["workspace_bytes"] == r256(n * dv * 4) + r256(n * 4)
+
+
+def test_plan_prefill(lib):
+    pl = binding.plan(2, 16, 1, 4096, 4096, 512, 512, num_sms=148)
+    assert pl["path"] == 0 and pl["dv_parts"] == 2 and pl["workspace_bytes"] == 0
+    assert pl["grid_ctas"] == 32 * 16 * 2 * 2
+    pl = binding.plan(1, 64, 8, 8192, 8192, 128, 128, num_sms=148)
+    assert pl["dv_parts"] == 1 and pl["grid_ctas"] == 64 * 64
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 16, 1, 1, 100, 512, 512), binding.ATTN_EINVAL),
+    ((1, 16, 3, 1, 100, 512, 512), binding.ATTN_EINVAL),       # Hq % Hkv != 0
+    ((1, 16, 1, 1, 0, 512, 512), binding.ATTN_EINVAL),         # no keys at all
+    ((1, 16, 1, 1, 100, 256, 256), binding.ATTN_EUNSUPPORTED),
+    ((1, 16, 1, 4, 100, 576, 512), binding.ATTN_EUNSUPPORTED),  # MLA shape is decode-only
+    ((1, 16, 1, 1, 100, 512, 128), binding.ATTN_EUNSUPPORTED),
+])
+def test_plan_rejects(lib, args, code):
+    pl = binding.Plan()
+    assert lib.attn_plan(*args, 0, 148, ctypes.byref(pl)) == code
+    assert binding.workspace_bytes(*args) == 0
+
+
+def _call(lib, **over):
+    """attn_fwd with fake but well-formed arguments; every case below must be
+    rejected before any CUDA work, so the fake pointers are never used."""
+    a = dict(q=0x10000, k=0x20000, v=0x30000, out=0x40000, lse=None, B=2, Hq=16, Hkv=1, Sq=1,
+             skv=0x50000, max_skv=256, d_k=512, d_v=512, scale=0.04, causal=1, dtype=0,
+             sq=binding.Strides(16 * 512, 512, 512), sk=binding.Strides(256 * 512, 256 * 512, 512),
+             sv=binding.Strides(256 * 512, 256 * 512, 512), so=binding.Strides(16 * 512, 512, 512),
+             ws=0x60000, ws_n=1 << 30, stream=None)
+    a.update(over)
+    return binding.fwd_raw(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                           a["Sq"], a["skv"], a["max_skv"], a["d_k"], a["d_v"], a["scale"],
+                           a["causal"], a["dtype"], a["sq"], a["sk"], a["sv"], a["so"], a["ws"],
+                           a["ws_n"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), binding.ATTN_EINVAL),
+    (dict(skv=None), binding.ATTN_EINVAL),
+    (dict(k=0x20008), binding.ATTN_EINVAL),                         # not 16-byte aligned
+    (dict(sk=binding.Strides(256 * 512, 256 * 512, 516)), binding.ATTN_EINVAL),  # stride % 8
+    (dict(sv=binding.Strides(-8, 0, 512)), binding.ATTN_EINVAL),
+    (dict(causal=2), binding.ATTN_EINVAL),
+    (dict(scale=float("nan")), binding.ATTN_EINVAL),
+    (dict(Hkv=3), binding.ATTN_EINVAL),
+    (dict(dtype=7), binding.ATTN_EINVAL),
+    (dict(d_k=64, d_v=64), binding.ATTN_EUNSUPPORTED),
+    (dict(ws=None), binding.ATTN_EWORKSPACE),
+    (dict(ws_n=64), binding.ATTN_EWORKSPACE),
+    (dict(ws=0x60004), binding.ATTN_EWORKSPACE),
+])
+def test_fwd_rejects_before_launch(lib, over, code):
+    assert _call(lib, **over) == code
