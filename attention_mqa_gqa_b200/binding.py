@@ -40,8 +40,8 @@ class AttnError(RuntimeError):
 
 
 # Every symbol include/attn_b200.h declares (checked by the CPU test suite).
-EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_last_device_error",
-           "attn_status_str", "attn_version")
+EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
+           "attn_decode_combine", "attn_last_device_error", "attn_status_str", "attn_version")
 
 _lib = None
 
@@ -61,10 +61,10 @@ def load(path: str | None = None):
     lib.attn_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(Plan)]
     lib.attn_workspace_bytes.restype = sz
     lib.attn_workspace_bytes.argtypes = [i32] * 7
-    lib.attn_fwd.restype = i32
-    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
-                             ctypes.c_float, i32, i32, Strides, Strides, Strides, Strides,
-                             vp, sz, vp]
+    for fn in (lib.attn_fwd, lib.attn_decode_partial, lib.attn_decode_combine):
+        fn.restype = i32
+        fn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
+                       ctypes.c_float, i32, i32, Strides, Strides, Strides, Strides, vp, sz, vp]
     lib.attn_last_device_error.restype = i32
     lib.attn_last_device_error.argtypes = [vp]
     lib.attn_status_str.restype = ctypes.c_char_p
@@ -112,11 +112,13 @@ def _strides4(t: torch.Tensor) -> Strides:
 
 def fwd_raw(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v, scale, causal,
             dtype_code_, sq: Strides, sk: Strides, sv: Strides, so: Strides,
-            workspace_ptr, workspace_nbytes, stream_ptr) -> int:
-    """Direct call with raw pointers (ints); returns the status code."""
-    return load().attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v,
-                           float(scale), int(causal), dtype_code_, sq, sk, sv, so,
-                           workspace_ptr, workspace_nbytes, stream_ptr)
+            workspace_ptr, workspace_nbytes, stream_ptr, entry: str = "attn_fwd") -> int:
+    """Direct call with raw pointers (ints); returns the status code.
+    ``entry`` selects attn_fwd, attn_decode_partial or attn_decode_combine."""
+    fn = getattr(load(), entry)
+    return fn(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v, float(scale),
+              int(causal), dtype_code_, sq, sk, sv, so, workspace_ptr, workspace_nbytes,
+              stream_ptr)
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -136,18 +136,24 @@ void set_smem(K kernel, int bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
+
 template <int DK, int DV, int NH, bool BF16>
 attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
-                            const attn_plan_t& pl, cudaStream_t st) {
+                            const attn_plan_t& pl, cudaStream_t st, int phases) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
-  auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
-  set_smem(kern, Tr::SMEM_BYTES);
-  dim3 grid(pl.head_blocks * pl.num_splits, dp.B, dp.Hkv);
-  kern<<<grid, 192, Tr::SMEM_BYTES, st>>>(mk, mv, dp);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-  attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  if (phases & PHASE_PARTIAL) {
+    auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
+    set_smem(kern, Tr::SMEM_BYTES);
+    dim3 grid(pl.head_blocks * pl.num_splits, dp.B, dp.Hkv);
+    kern<<<grid, 192, Tr::SMEM_BYTES, st>>>(mk, mv, dp);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  }
+  if (phases & PHASE_COMBINE) {
+    attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  }
   return ATTN_OK;
 }
 
@@ -178,12 +184,16 @@ size_t attn_workspace_bytes(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k
   return pl.workspace_bytes;
 }
 
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+}  // extern "C"
+
+namespace {
+
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse,
                        int B, int Hq, int Hkv, int Sq, const int32_t* skv_per_seq, int max_skv,
                        int d_k, int d_v, float scale, int causal, attn_dtype_t dtype,
                        attn_strides_t sq, attn_strides_t sk, attn_strides_t sv,
                        attn_strides_t so, void* workspace, size_t workspace_bytes,
-                       void* cuda_stream) {
+                       void* cuda_stream, int phases) {
   // ---- validation (nothing touches the GPU before this passes)
   if (!q || !k || !v || !out || !skv_per_seq) return ATTN_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_EINVAL;
@@ -195,6 +205,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
   attn_plan_t pl;
   attn_status_t rc = plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype, 0, &pl);
   if (rc != ATTN_OK) return rc;
+  if (phases != PHASE_ALL && pl.path != 1) return ATTN_EINVAL;  // phases exist for decode only
   if ((Sq > 1 && sq.s == 0) || sk.s == 0 || sv.s == 0 || (Sq > 1 && so.s == 0)) return ATTN_EINVAL;
   if (pl.workspace_bytes > 0) {
     if (!workspace || !aligned16(workspace)) return ATTN_EWORKSPACE;
@@ -243,13 +254,13 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     cp.num_splits = pl.num_splits;
     cp.split_tokens = pl.split_tokens;
     if (d_k == 128)
-      return bf16 ? launch_decode<128, 128, 16, true>(mk, mv, dp, cp, pl, st)
-                  : launch_decode<128, 128, 16, false>(mk, mv, dp, cp, pl, st);
+      return bf16 ? launch_decode<128, 128, 16, true>(mk, mv, dp, cp, pl, st, phases)
+                  : launch_decode<128, 128, 16, false>(mk, mv, dp, cp, pl, st, phases);
     if (d_k == 512)
-      return bf16 ? launch_decode<512, 512, 16, true>(mk, mv, dp, cp, pl, st)
-                  : launch_decode<512, 512, 16, false>(mk, mv, dp, cp, pl, st);
-    return bf16 ? launch_decode<576, 512, 64, true>(mk, mv, dp, cp, pl, st)
-                : launch_decode<576, 512, 64, false>(mk, mv, dp, cp, pl, st);
+      return bf16 ? launch_decode<512, 512, 16, true>(mk, mv, dp, cp, pl, st, phases)
+                  : launch_decode<512, 512, 16, false>(mk, mv, dp, cp, pl, st, phases);
+    return bf16 ? launch_decode<576, 512, 64, true>(mk, mv, dp, cp, pl, st, phases)
+                : launch_decode<576, 512, 64, false>(mk, mv, dp, cp, pl, st, phases);
   }
 
   CUtensorMap mq;
@@ -276,6 +287,41 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
                 : launch_prefill<128, 128, false>(mq, mk, mv, pp, pl, st);
   return bf16 ? launch_prefill<512, 256, true>(mq, mk, mv, pp, pl, st)
               : launch_prefill<512, 256, false>(mq, mk, mv, pp, pl, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+#define ATTN_FWD_ARGS                                                                           \
+  q, k, v, out, lse, B, Hq, Hkv, Sq, skv_per_seq, max_skv, d_k, d_v, scale, causal, dtype, sq, \
+      sk, sv, so, workspace, workspace_bytes, cuda_stream
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Sq, const int32_t* skv_per_seq, int max_skv,
+                       int d_k, int d_v, float scale, int causal, attn_dtype_t dtype,
+                       attn_strides_t sq, attn_strides_t sk, attn_strides_t sv,
+                       attn_strides_t so, void* workspace, size_t workspace_bytes,
+                       void* cuda_stream) {
+  return fwd_impl(ATTN_FWD_ARGS, PHASE_ALL);
+}
+
+attn_status_t attn_decode_partial(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int B, int Hq, int Hkv, int Sq,
+                                  const int32_t* skv_per_seq, int max_skv, int d_k, int d_v,
+                                  float scale, int causal, attn_dtype_t dtype, attn_strides_t sq,
+                                  attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                                  void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return fwd_impl(ATTN_FWD_ARGS, PHASE_PARTIAL);
+}
+
+attn_status_t attn_decode_combine(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int B, int Hq, int Hkv, int Sq,
+                                  const int32_t* skv_per_seq, int max_skv, int d_k, int d_v,
+                                  float scale, int causal, attn_dtype_t dtype, attn_strides_t sq,
+                                  attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                                  void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return fwd_impl(ATTN_FWD_ARGS, PHASE_COMBINE);
 }
 
 attn_status_t attn_last_device_error(void* cuda_stream) {

@@ -1,0 +1,568 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 attention library (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload: MQA decode at head_dim 512 (B=32, Hq=16, Hkv=1, per-sequence
+KV length uniform in [1024, 8192], bf16): one step = one decode forward of
+the whole batch (split-KV partial kernel + LSE combine).  The metric is the
+KV-cache bytes read per second (each cached K/V byte counted once).  The
+same line carries, measured in the same run, the d=512 MQA causal prefill
+(B=2, Hq=16, S=4096) in TFLOP/s, the roofline fraction of the dominant
+kernel against the measured peaks, the CPU oracle's throughput on a bounded
+sample, and an end-to-end figure through the C ABI with host buffers.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and cudaDeviceSynchronize on both sides; CUDA events on the launching stream;
+with N GPUs (torchrun) every rank runs its own replica of the workload and
+the time is the max over ranks.  Inputs are larger than L2 for the decode
+workloads (the KV cache alone is 302 MB vs 126 MB L2).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_mqa_gqa_b200 import workloads as wl  # noqa: E402
+
+KERNEL_SOURCES = ["attention_mqa_gqa_b200/csrc/sm100.cuh", "attention_mqa_gqa_b200/csrc/decode_kernel.cuh",
+                  "attention_mqa_gqa_b200/csrc/prefill_kernel.cuh", "attention_mqa_gqa_b200/csrc/attn_api.cu"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- accounting
+
+def kv_bytes(w, skv) -> int:
+    """Cached K/V bytes one decode step must read: every key row of every
+    sequence once (MLA: the 576-wide row once, V aliases its first 512)."""
+    n = int(sum(int(x) for x in skv))
+    el = 2
+    if w.mla:
+        return n * w.d_k * el
+    return n * w.Hkv * (w.d_k + w.d_v) * el
+
+
+def visible_pairs(w, skv) -> int:
+    """Number of (query row, key) pairs the softmax covers, over all heads.
+    Causal rows are bottom-right aligned: row i of Sq sees
+    max(0, i + L - Sq + 1) of a sequence's L keys, so the last min(Sq, L)
+    rows see L - c + 1 .. L keys (c = that count)."""
+    tot = 0
+    for L in skv:
+        L = int(L)
+        if not w.causal:
+            tot += w.Sq * L
+        else:
+            c = min(w.Sq, L)
+            tot += (2 * L - c + 1) * c // 2
+    return tot * w.Hq
+
+
+def flops(w, skv) -> int:
+    return 2 * (w.d_k + w.d_v) * visible_pairs(w, skv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    for s in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("sources_sha") != sources_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.id = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.id:
+                cmd += ["--id", self.id]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.02)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return None
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+class GpuRunner:
+    """Holds one workload's device tensors and launches steps through the C ABI."""
+
+    def __init__(self, w, inp, device):
+        from attention_mqa_gqa_b200 import binding
+
+        self.b = binding
+        self.w = w
+        self.dev = device
+        self.skv_host = inp["skv"]
+        self.max_skv = inp["max_skv"]
+        self.q = inp["q"].to(device)
+        if w.mla:
+            cache = inp["cache"].to(device)
+            B, S, dk = cache.shape
+            self.k = cache.view(B, 1, S, dk)
+            self.v = cache.view(B, 1, S, dk)[..., : w.d_v]
+            self._keep = cache
+        else:
+            self.k = inp["k"].to(device)
+            self.v = inp["v"].to(device)
+        self.skv = inp["skv"].to(device)
+        self.out = torch.empty(w.B, w.Hq, w.Sq, w.d_v, dtype=w.dtype, device=device)
+        self.lse = torch.empty(w.B, w.Hq, w.Sq, dtype=torch.float32, device=device)
+        nws = binding.workspace_bytes(w.B, w.Hq, w.Hkv, w.Sq, self.max_skv, w.d_k, w.d_v)
+        self.ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=device)
+        self.plan = binding.plan(w.B, w.Hq, w.Hkv, w.Sq, self.max_skv, w.d_k, w.d_v, w.dtype)
+        self.stream = torch.cuda.current_stream(device)
+        self._args = None
+
+    def args(self):
+        if self._args is None:
+            b, w = self.b, self.w
+            st = lambda t: b.Strides(t.stride(0), t.stride(1), t.stride(2))
+            self._args = (self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                          self.out.data_ptr(), self.lse.data_ptr(), w.B, w.Hq, w.Hkv, w.Sq,
+                          self.skv.data_ptr(), self.max_skv, w.d_k, w.d_v, w.scale,
+                          int(w.causal), b.dtype_code(w.dtype), st(self.q), st(self.k),
+                          st(self.v), st(self.out), self.ws.data_ptr(), self.ws.numel(),
+                          self.stream.cuda_stream)
+        return self._args
+
+    def call(self, entry="attn_fwd"):
+        rc = self.b.fwd_raw(*self.args(), entry=entry)
+        if rc != 0:
+            raise self.b.AttnError(rc, entry)
+
+    @property
+    def decode(self):
+        return self.plan["path"] == 1
+
+    def launches_per_step(self):
+        return 2 if self.decode else 1
+
+    def timed(self, steps, warmup, events_per_kernel=True):
+        """Run warmup + steps; return (total_ms, dominant kernel mean ms,
+        other kernel mean ms)."""
+        for _ in range(warmup):
+            self.call()
+        torch.cuda.synchronize(self.dev)
+        E = lambda: torch.cuda.Event(enable_timing=True)
+        if self.decode and events_per_kernel:
+            ev = [E() for _ in range(2 * steps + 1)]
+            start, end = ev[0], ev[-1]
+            torch.cuda.synchronize(self.dev)
+            ev[0].record(self.stream)
+            for i in range(steps):
+                self.call("attn_decode_partial")
+                ev[2 * i + 1].record(self.stream)
+                self.call("attn_decode_combine")
+                ev[2 * i + 2].record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            part = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
+            comb = [ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(steps)]
+            return start.elapsed_time(end), statistics.mean(part), statistics.mean(comb)
+        ev = [E() for _ in range(steps + 1)]
+        torch.cuda.synchronize(self.dev)
+        ev[0].record(self.stream)
+        for i in range(steps):
+            self.call()
+            ev[i + 1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+        return ev[0].elapsed_time(ev[-1]), statistics.mean(per), 0.0
+
+    def e2e(self, steps, warmup, inp):
+        """Same step through the C ABI with the step's inputs in pinned host
+        memory: H2D copy of the inputs, the forward, D2H copy of out and lse,
+        synchronised every step.  Decode keeps the KV cache resident (it is
+        state, not a per-step input); prefill copies q, k and v every step."""
+        pin = lambda t: t.pin_memory()
+        hq = pin(inp["q"])
+        hskv = pin(inp["skv"])
+        hk = hv = None
+        if not self.decode:  # prefill shapes have separate K and V tensors
+            hk, hv = pin(inp["k"]), pin(inp["v"])
+        hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        hlse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        h2d = hq.numel() * hq.element_size() + hskv.numel() * 4
+        if hk is not None:
+            h2d += hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+
+        def step():
+            self.q.copy_(hq, non_blocking=True)
+            self.skv.copy_(hskv, non_blocking=True)
+            if hk is not None:
+                self.k.copy_(hk, non_blocking=True)
+                self.v.copy_(hv, non_blocking=True)
+            self.call()
+            hout.copy_(self.out, non_blocking=True)
+            hlse.copy_(self.lse, non_blocking=True)
+            self.stream.synchronize()
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(self.dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        for _ in range(steps):
+            step()
+        b_.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return a.elapsed_time(b_), h2d, d2h
+
+
+def metric_of(w):
+    if w.is_decode:
+        return "kv_cache_read_GBps", "GB/s", True
+    return "attention_TFLOPs", "TFLOP/s", True
+
+
+def value_of(w, skv, ms):
+    if w.is_decode:
+        return kv_bytes(w, skv) / (ms * 1e-3) / 1e9
+    return flops(w, skv) / (ms * 1e-3) / 1e12
+
+
+def roofline(w, skv, kernel_ms, peaks, peak_src, long_run, traffic):
+    if w.is_decode:
+        achieved = kv_bytes(w, skv) / (kernel_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"hbm_gbs ({peak_src})"}
+    key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
+    peak = float(peaks[key])
+    if w.dtype == torch.float16:
+        key += " (fp16 = bf16 dense rate)"
+    achieved = flops(w, skv) / (kernel_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{key} ({peak_src})"}
+
+
+def config_of(w, inp, parallelism):
+    skv = inp["skv"]
+    d = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "d_k": w.d_k,
+         "d_v": w.d_v, "causal": w.causal, "scale": round(w.scale, 6), "mla_absorbed": w.mla,
+         "skv": f"U[{w.skv_lo},{w.skv_hi}] seed {w.seed}" if w.skv_lo != w.skv_hi else w.skv_lo,
+         "skv_total": int(skv.sum()), "parallelism": parallelism}
+    if w.is_decode:
+        d["l2"] = f"inputs larger than L2: KV {kv_bytes(w, skv) / 1e6:.0f} MB > 126 MB"
+    else:
+        qb = w.B * w.Hq * w.Sq * w.d_k * 2
+        d["l2"] = (f"no flush: Q {qb / 1e6:.0f} MB and O stream through; K/V "
+                   f"{kv_bytes(w, skv) / 1e6:.1f} MB are meant to stay in L2 (prefill reuses them)")
+    return d
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, inp, budget_s):
+    """The first n sequences (all heads) whose estimated oracle cost fits the
+    budget (the fp64 C oracle runs at roughly 1 GFLOP/s per thread)."""
+    rate = 1.0e9 * (os.cpu_count() or 1)
+    skv = inp["skv"].tolist()
+    n, acc = 0, 0.0
+    for b in range(w.B):
+        cost = flops(w.scaled(B=1), [skv[b]]) / rate
+        if n > 0 and acc + cost > budget_s:
+            break
+        n += 1
+        acc += cost
+    return n
+
+
+def run_oracle(w, inp, n):
+    from oracle import c_oracle
+
+    t0 = time.perf_counter()
+    c_oracle.attention_fwd(inp["q"][:n], inp["k"][:n], inp["v"][:n], inp["skv"][:n].tolist(),
+                           w.scale, w.causal)
+    return time.perf_counter() - t0
+
+
+def cpu_value(w, inp, n, secs):
+    skv = inp["skv"][:n].tolist()
+    wb = w.scaled(B=n)
+    if w.is_decode:
+        return kv_bytes(wb, skv) / secs / 1e9
+    return flops(wb, skv) / secs / 1e12
+
+
+# ----------------------------------------------------------------- main
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def allreduce(x, op, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def reference_arm(args, world, rank):
+    """The oracle as it stands, timed on the host cores; rank 0 only."""
+    if rank != 0:
+        return 0
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w)
+    n = oracle_sample(w, inp, budget_s=args.ref_step_budget)
+    from oracle import c_oracle
+
+    c_oracle.build()
+    for _ in range(args.warmup):
+        run_oracle(w, inp, n)
+    t = 0.0
+    for _ in range(args.steps):
+        t += run_oracle(w, inp, n)
+    val = cpu_value(w, inp, n, t / args.steps)
+    metric, unit, hib = metric_of(w)
+    cores = os.cpu_count() or 1
+    sample = f"first {n} of {w.B} sequences, all {w.Hq} heads, per step"
+    line = {"impl": "reference", "metric": f"{w.name}_{metric}", "value": round(val, 4),
+            "unit": unit, "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": hib,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, inp, "host cores"),
+            "cpu_baseline": {"value": round(val, 4), "unit": unit, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_workload(w, inp, device, steps, warmup, world):
+    g = GpuRunner(w, inp, device)
+    if steps is None:  # size the timed region to about 2 s
+        t_ms, _, _ = g.timed(5, 3, events_per_kernel=False)
+        steps = int(min(20000, max(20, 2000.0 / max(t_ms / 5, 1e-3))))
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    total_ms, k_ms, other_ms = g.timed(steps, warmup)
+    clocks = sampler.stop()
+    barrier(world)
+    return g, steps, total_ms, k_ms, other_ms, clocks
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mqa_decode", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill figure")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--ref-step-budget", type=float, default=2.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        rc = reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return rc
+
+    from attention_mqa_gqa_b200 import binding, build
+
+    if not os.path.exists(binding.LIB_PATH):
+        build.build()
+    binding.load()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+
+    w = wl.WORKLOADS[args.workload]
+    if rank:
+        w = w.scaled(seed=w.seed + 1000 * rank)  # each replica its own batch
+    inp = wl.make_inputs(w)
+    g, steps, total_ms, k_ms, other_ms, clocks = measure_workload(w, inp, device, args.steps,
+                                                                  args.warmup, world)
+    import torch.distributed as dist_mod
+
+    max_ms = allreduce(total_ms, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
+    work = kv_bytes(w, inp["skv"]) if w.is_decode else flops(w, inp["skv"])
+    work_all = allreduce(work, dist_mod.ReduceOp.SUM if world > 1 else None, world, device)
+    ms_step = max_ms / steps
+    scale_div = 1e9 if w.is_decode else 1e12
+    value = work_all * steps / (max_ms * 1e-3) / scale_div
+    metric, unit, hib = metric_of(w)
+    long_run = total_ms > 1000.0
+    kname = "decode_split_kernel" if g.decode else "prefill_kernel"
+    roof = roofline(w, inp["skv"], k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
+    roof["kernel"] = kname
+    roof["kernel_ms"] = round(k_ms, 5)
+    if g.decode:
+        roof["combine_ms"] = round(other_ms, 5)
+
+    # end to end through the C ABI with host buffers
+    e2e_steps = max(10, min(steps, 200))
+    e_ms, h2d, d2h = g.e2e(e2e_steps, 3, inp)
+    e_ms = allreduce(e_ms, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
+    e_val = work_all * e2e_steps / (e_ms * 1e-3) / scale_div
+    assert binding.last_device_error() == binding.ATTN_OK, "device-side wait timed out"
+
+    line = {"metric": f"{w.name}_{metric}", "value": round(value, 3), "unit": unit,
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 5), "higher_is_better": hib, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "fp16",
+            "data": "synthetic (seeded N(0,1), rounded once to the element type)",
+            "config": config_of(w, inp, f"replicas x{world}" if world > 1 else "single GPU"),
+            "roofline": roof, "gpu_launches": g.launches_per_step() * steps,
+            "clocks": clocks,
+            "e2e": {"value": round(e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps}}
+    del g
+
+    # secondary figure: d=512 MQA causal prefill (B=2, Hq=16, S=4096)
+    if not args.no_secondary and args.workload == "mqa_decode":
+        w2 = wl.WORKLOADS["mqa_prefill"]
+        if rank:
+            w2 = w2.scaled(seed=w2.seed + 1000 * rank)
+        inp2 = wl.make_inputs(w2)
+        g2, steps2, tot2, k2, _, clocks2 = measure_workload(w2, inp2, device, args.steps,
+                                                            args.warmup, world)
+        max2 = allreduce(tot2, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
+        work2 = allreduce(flops(w2, inp2["skv"]), dist_mod.ReduceOp.SUM if world > 1 else None,
+                          world, device)
+        r2 = roofline(w2, inp2["skv"], k2, peaks, peak_src, tot2 > 1000.0,
+                      traffic_for("prefill_kernel", w2.name))
+        r2["kernel"] = "prefill_kernel"
+        line["prefill"] = {"metric": f"{w2.name}_attention_TFLOPs",
+                           "value": round(work2 * steps2 / (max2 * 1e-3) / 1e12, 2),
+                           "unit": "TFLOP/s", "steps": steps2, "ms_per_step": round(max2 / steps2, 4),
+                           "config": config_of(w2, inp2, "single GPU" if world == 1 else f"replicas x{world}"),
+                           "roofline": r2, "clocks": clocks2}
+        del g2
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n = oracle_sample(w, inp, budget_s=15.0)
+        from oracle import c_oracle
+
+        c_oracle.build()
+        secs = run_oracle(w, inp, n)
+        line["cpu_baseline"] = {"value": round(cpu_value(w, inp, n, secs), 4), "unit": unit,
+                                "cores": os.cpu_count() or 1, "kind": "oracle",
+                                "sample": f"first {n} of {w.B} sequences, all {w.Hq} heads "
+                                          f"({secs:.1f} s, fp64 C oracle)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -120,6 +120,33 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
                        void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * The two steps attn_fwd enqueues for a decode problem (Sq == 1), callable
+ * separately with attn_fwd's arguments (for timing each kernel, or for
+ * overlapping the merge with other work):
+ *   attn_decode_partial  -- every (sequence, kv head, head block, KV split)
+ *                           attends over its keys and writes a normalised
+ *                           partial output and its LSE into the workspace;
+ *   attn_decode_combine  -- merges the splits of each (b, h) in split order:
+ *                           L = ln sum_s exp(lse_s), out = sum_s exp(lse_s - L) o_s
+ *                           ("GQA和MLA详解" section 4: a fixed reduction order keeps
+ *                           the result bitwise reproducible).
+ * Same validation and errors as attn_fwd; ATTN_EINVAL when Sq > 1.  The
+ * combine step reads what the partial step wrote into the same workspace.
+ */
+attn_status_t attn_decode_partial(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int B, int Hq, int Hkv, int Sq,
+                                  const int32_t* skv_per_seq, int max_skv, int d_k, int d_v,
+                                  float scale, int causal, attn_dtype_t dtype, attn_strides_t sq,
+                                  attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                                  void* workspace, size_t workspace_bytes, void* cuda_stream);
+attn_status_t attn_decode_combine(const void* q, const void* k, const void* v, void* out,
+                                  float* lse, int B, int Hq, int Hkv, int Sq,
+                                  const int32_t* skv_per_seq, int max_skv, int d_k, int d_v,
+                                  float scale, int causal, attn_dtype_t dtype, attn_strides_t sq,
+                                  attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                                  void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * error word.  ATTN_OK if no kernel of this library reported a problem
  * since the last call, ATTN_ETIMEOUT if a device-side wait gave up (the
