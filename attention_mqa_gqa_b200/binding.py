@@ -41,7 +41,9 @@ class AttnError(RuntimeError):
 
 # Every symbol include/attn_b200.h declares (checked by the CPU test suite).
 EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
-           "attn_decode_combine", "attn_last_device_error", "attn_status_str", "attn_version")
+           "attn_decode_combine", "attn_fwd_noalloc", "attn_last_device_error", "attn_status_str",
+           "attn_version")
+NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in the header
 
 _lib = None
 
@@ -65,6 +67,10 @@ def load(path: str | None = None):
         fn.restype = i32
         fn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
                        ctypes.c_float, i32, i32, Strides, Strides, Strides, Strides, vp, sz, vp]
+    lib.attn_fwd_noalloc.restype = i32
+    lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
+                                     ctypes.c_float, i32, i32, Strides, Strides, Strides,
+                                     Strides, vp]
     lib.attn_last_device_error.restype = i32
     lib.attn_last_device_error.argtypes = [vp]
     lib.attn_status_str.restype = ctypes.c_char_p
@@ -147,6 +153,29 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
                  ws_ptr, ws_n, st.cuda_stream)
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
+
+
+def attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                     skv: torch.Tensor, max_skv: int, scale: float, causal: bool = True,
+                     lse: torch.Tensor | None = None,
+                     stream: torch.cuda.Stream | None = None) -> None:
+    """Like :func:`attn_fwd` but without a workspace: the library's built-in
+    scratch buffer is used (for callers that cannot allocate device memory;
+    see the header).  Calls sharing the buffer must not overlap on the GPU."""
+    B, Hq, Sq, d_k = q.shape
+    Hkv, d_v = k.shape[1], v.shape[-1]
+    if skv.dtype != torch.int32:
+        raise TypeError("skv must be int32")
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise TypeError("lse must be a contiguous float32 tensor")
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = load().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq,
+                                 skv.data_ptr(), int(max_skv), d_k, d_v, float(scale), int(causal),
+                                 dtype_code(q.dtype), _strides4(q), _strides4(k), _strides4(v),
+                                 _strides4(out), st.cuda_stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_noalloc")
 
 
 def last_device_error(stream: torch.cuda.Stream | None = None) -> int:

@@ -350,3 +350,75 @@ const char* attn_status_str(attn_status_t s) {
 const char* attn_version(void) { return "0.1.0"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_fwd_noalloc: attn_fwd for callers that cannot allocate device memory.
+//
+// The decode path needs scratch memory (per-split partial outputs and LSEs)
+// that attn_fwd takes from a caller-provided workspace.  Some callers cannot
+// obtain one: a plugin run by a host framework that owns all device memory
+// and hands plugins no allocator, or a latency-critical loop where
+// cudaMalloc's implicit device-wide synchronisation is not acceptable.  This
+// entry point uses a fixed buffer compiled into the library instead.
+//
+// The buffer is a file-scope __device__ array of ATTN_NOALLOC_SCRATCH_BYTES;
+// every GPU that loads the library holds it until the process exits.  Host
+// code cannot pass the array's name to a kernel (on the host it only names a
+// stand-in object), so its device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, on the first call made on
+// that device.  All calls share the buffer and it keeps whatever the last
+// call left there; the kernels write every scratch value before reading it,
+// so nothing has to be cleared between calls.  Calls that overlap on the GPU
+// (other streams, other host threads) race on the buffer.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once).
+attn_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return ATTN_ECUDA; }
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return ATTN_ECUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                          float* lse, int B, int Hq, int Hkv, int Sq,
+                                          const int32_t* skv_per_seq, int max_skv, int d_k,
+                                          int d_v, float scale, int causal, attn_dtype_t dtype,
+                                          attn_strides_t sq, attn_strides_t sk,
+                                          attn_strides_t sv, attn_strides_t so,
+                                          void* cuda_stream) {
+  // Size check first: a problem whose scratch would not fit is refused
+  // before anything touches the device.
+  attn_plan_t pl;
+  attn_status_t rc = plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype, 0, &pl);
+  if (rc != ATTN_OK) return rc;
+  if (pl.workspace_bytes > (size_t)ATTN_NOALLOC_SCRATCH_BYTES) return ATTN_EWORKSPACE;
+  void* scratch = nullptr;
+  if (pl.workspace_bytes > 0) {
+    rc = noalloc_scratch(&scratch);
+    if (rc != ATTN_OK) return rc;
+  }
+  return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_per_seq, max_skv, d_k, d_v, scale,
+                  causal, dtype, sq, sk, sv, so, scratch, (size_t)ATTN_NOALLOC_SCRATCH_BYTES,
+                  cuda_stream, PHASE_ALL);
+}

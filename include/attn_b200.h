@@ -147,6 +147,32 @@ attn_status_t attn_decode_combine(const void* q, const void* k, const void* v, v
                                   void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * attn_fwd without a workspace argument, for callers that cannot allocate
+ * device memory (the pages have no counterpart: this is a library concern).
+ * Examples: a plugin run by a host framework that owns all device memory
+ * and gives plugins no allocator, or a latency-critical loop in which
+ * cudaMalloc's implicit device-wide synchronisation is not acceptable.
+ *
+ * Scratch comes from a buffer of ATTN_NOALLOC_SCRATCH_BYTES compiled into
+ * the library (held on every GPU that loads the library until the process
+ * exits); the call itself allocates nothing.  Problems whose scratch
+ * (attn_workspace_bytes) exceeds that size return ATTN_EWORKSPACE before
+ * anything is enqueued.  The first call on each device looks up the
+ * buffer's device address (cudaGetSymbolAddress, that device current); make
+ * that first call before any stream capture.  All calls share the buffer:
+ * calls that overlap on the GPU (concurrent streams or host threads) race,
+ * so serialise them.  Otherwise the same arguments, semantics and errors as
+ * attn_fwd.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                               float* lse, int B, int Hq, int Hkv, int Sq,
+                               const int32_t* skv_per_seq, int max_skv, int d_k, int d_v,
+                               float scale, int causal, attn_dtype_t dtype, attn_strides_t sq,
+                               attn_strides_t sk, attn_strides_t sv, attn_strides_t so,
+                               void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * error word.  ATTN_OK if no kernel of this library reported a problem
  * since the last call, ATTN_ETIMEOUT if a device-side wait gave up (the
