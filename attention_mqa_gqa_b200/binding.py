@@ -25,8 +25,8 @@ class Strides(ctypes.Structure):
 
 class Plan(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
-                ("head_blocks", ctypes.c_int), ("num_splits", ctypes.c_int),
-                ("split_tokens", ctypes.c_int), ("dv_parts", ctypes.c_int),
+                ("head_blocks", ctypes.c_int), ("kv_ranges", ctypes.c_int),
+                ("partials", ctypes.c_int64), ("dv_parts", ctypes.c_int),
                 ("grid_ctas", ctypes.c_int64), ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self) -> dict:

@@ -19,7 +19,6 @@
 namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
-constexpr int kDecodeTile = 128;
 
 // ------------------------------------------------------------------ driver
 
@@ -63,6 +62,25 @@ bool make_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, u
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over q [B, Hq, 1, D] seen as rows (head) of D columns: box = 64
+// columns x `rows` heads, 128-byte swizzle (the decode kernel's Q^T chunks).
+bool make_q_rows_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t H,
+                     uint64_t B, int64_t sh, int64_t sb, uint32_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  if (H == 1) sh = (int64_t)D;
+  if (B == 1) sb = sh * (int64_t)H;
+  cuuint64_t dims[3] = {D, H, B};
+  cuuint64_t strides[2] = {(cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  cuuint32_t box[3] = {64, rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
@@ -78,6 +96,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool strides_ok(const attn_strides_t& s) {
   return s.b >= 0 && s.h >= 0 && s.s >= 0 && s.b % 8 == 0 && s.h % 8 == 0 && s.s % 8 == 0;
 }
+
+// Resident decode CTAs per SM (must match DecodeTraits<...>::CTAS).
+int decode_ctas_per_sm(int d_k) { return d_k == 128 ? 2 : 1; }
 
 bool shape_supported(int Sq, int d_k, int d_v) {
   if (Sq > 1) return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512);
@@ -110,22 +131,15 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
   const int NH = d_k == 576 ? 64 : 16;
   pl->heads_per_cta = NH;
   pl->head_blocks = (G + NH - 1) / NH;
-  const int64_t units = (int64_t)B * Hkv * pl->head_blocks;
-  const int tiles = (max_skv + kDecodeTile - 1) / kDecodeTile;
-  const int ctas_per_sm = d_k == 576 ? 1 : 2;
-  // Aim for about three resident waves of CTAs so the ragged per-sequence
-  // lengths (unknown to the host) even out across the SMs.
-  const int64_t target = (int64_t)num_sms * ctas_per_sm * 3;
-  int64_t want = (target + units - 1) / units;
-  if (want < 1) want = 1;
-  int split_tiles = (int)((tiles + want - 1) / want);
-  if (split_tiles < 1) split_tiles = 1;
-  pl->split_tokens = split_tiles * kDecodeTile;
-  pl->num_splits = (tiles + split_tiles - 1) / split_tiles;
-  pl->grid_ctas = units * pl->num_splits;
-  if (B > 65535 || Hkv > 65535 || (int64_t)pl->head_blocks * pl->num_splits > 0x7fffffffLL)
-    return ATTN_EUNSUPPORTED;
-  const size_t n = (size_t)B * Hq * pl->num_splits;
+  // One persistent wave: every SM runs decode_ctas_per_sm(d_k) CTAs; the
+  // key tiles are cut into equal ranges, one per CTA of each head block.
+  int ranges = num_sms * decode_ctas_per_sm(d_k) / pl->head_blocks;
+  if (ranges < 1) ranges = 1;
+  pl->kv_ranges = ranges;
+  pl->partials = (int64_t)ranges + (int64_t)B * Hkv;
+  pl->grid_ctas = (int64_t)ranges * pl->head_blocks;
+  if (pl->grid_ctas > 0x7fffffffLL || (int64_t)B * Hq > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
+  const size_t n = (size_t)pl->partials * G;
   pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float));
   return ATTN_OK;
 }
@@ -139,15 +153,15 @@ void set_smem(K kernel, int bytes) {
 enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
 
 template <int DK, int DV, int NH, bool BF16>
-attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
+attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
                             const attn_plan_t& pl, cudaStream_t st, int phases) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
+  static_assert(Tr::CTAS == (DK == 128 ? 2 : 1), "decode_ctas_per_sm out of sync");
   if (phases & PHASE_PARTIAL) {
     auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
     set_smem(kern, Tr::SMEM_BYTES);
-    dim3 grid(pl.head_blocks * pl.num_splits, dp.B, dp.Hkv);
-    kern<<<grid, 192, Tr::SMEM_BYTES, st>>>(mk, mv, dp);
+    kern<<<(unsigned)pl.grid_ctas, 192, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   if (phases & PHASE_COMBINE) {
@@ -222,12 +236,13 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   if (!make_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b)) return ATTN_ECUDA;
 
   if (pl.path == 1) {
+    if ((Hq > 1 && sq.h == 0) || (B > 1 && sq.b == 0)) return ATTN_EINVAL;
+    CUtensorMap mq;
+    if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, (uint32_t)pl.heads_per_cta))
+      return ATTN_ECUDA;
     attn::DecodeParams dp{};
-    dp.q = q;
-    dp.q_sb = sq.b;
-    dp.q_sh = sq.h;
     dp.skv = skv_per_seq;
-    const size_t n = (size_t)B * Hq * pl.num_splits;
+    const size_t n = (size_t)pl.partials * G;
     dp.ws_o = reinterpret_cast<float*>(workspace);
     dp.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                          align256(n * d_v * sizeof(float)));
@@ -235,8 +250,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     dp.Hq = Hq;
     dp.Hkv = Hkv;
     dp.G = G;
-    dp.num_splits = pl.num_splits;
-    dp.split_tiles = pl.split_tokens / kDecodeTile;
+    dp.ranges = pl.kv_ranges;
     dp.head_blocks = pl.head_blocks;
     dp.scale_log2 = scale_log2;
     dp.timeout_ns = kDefaultTimeoutNs;
@@ -250,17 +264,18 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     cp.lse = lse;
     cp.B = B;
     cp.Hq = Hq;
+    cp.Hkv = Hkv;
+    cp.G = G;
     cp.DV = d_v;
-    cp.num_splits = pl.num_splits;
-    cp.split_tokens = pl.split_tokens;
+    cp.ranges = pl.kv_ranges;
     if (d_k == 128)
-      return bf16 ? launch_decode<128, 128, 16, true>(mk, mv, dp, cp, pl, st, phases)
-                  : launch_decode<128, 128, 16, false>(mk, mv, dp, cp, pl, st, phases);
+      return bf16 ? launch_decode<128, 128, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
+                  : launch_decode<128, 128, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
     if (d_k == 512)
-      return bf16 ? launch_decode<512, 512, 16, true>(mk, mv, dp, cp, pl, st, phases)
-                  : launch_decode<512, 512, 16, false>(mk, mv, dp, cp, pl, st, phases);
-    return bf16 ? launch_decode<576, 512, 64, true>(mk, mv, dp, cp, pl, st, phases)
-                : launch_decode<576, 512, 64, false>(mk, mv, dp, cp, pl, st, phases);
+      return bf16 ? launch_decode<512, 512, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
+                  : launch_decode<512, 512, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
+    return bf16 ? launch_decode<576, 512, 64, true>(mq, mk, mv, dp, cp, pl, st, phases)
+                : launch_decode<576, 512, 64, false>(mq, mk, mv, dp, cp, pl, st, phases);
   }
 
   CUtensorMap mq;

@@ -1,28 +1,37 @@
-// decode_kernel.cuh -- split-KV decode (one query row per head, Sq == 1).
+// decode_kernel.cuh -- persistent split-KV decode (one query row per head,
+// Sq == 1) and the LSE combine.
 //
 // Decode reads the whole KV cache once per step and is bandwidth-bound
-// ("GQA和MLA详解" section 1; "Full 路线" section 4.5).  Every KV byte must
-// therefore be read from HBM once for all G query heads that share it
+// ("GQA和MLA详解" section 1; "Full 路线" section 4.5), so every K/V byte
+// must be read from HBM once for all G query heads that share it
 // ("GQA和MLA详解" section 2: real kernels index the shared head instead of
 // copying it).  This kernel puts 128 keys of one KV head in the MMA M
-// dimension and the group's query heads in N ("keys x heads" orientation):
+// dimension and the group's query heads in N:
 //
 //   S^T[128 keys x NH heads] = K_tile[128 x d_k] * Q^T          (tcgen05, TMEM)
-//   softmax over keys per head (online, with a lazily updated max)
+//   softmax over keys per head (online, with a lazily raised max)
 //   O^T[d_v x NH]           += V_tile^T[d_v x 128] * P^T[128 x NH]
 //
-// so G = 16 MQA heads, G = 8 GQA heads (padded to 16) and 64 of the 128 MLA
-// heads are MMA-efficient without padding M.  Each CTA handles one
-// (batch, kv head, head block, KV split); partial outputs (normalised) and
-// their LSEs go to the workspace and a combine kernel merges the splits.
+// so 16 MQA heads, 8 GQA heads (padded to 16) and 64 of the 128 MLA heads
+// use the tensor cores without padding M with absent query rows.
+//
+// Scheduling: the grid is persistent (one wave).  The key tiles of all
+// (sequence, kv head) units, laid end to end, are cut into `ranges` equal
+// contiguous ranges; each CTA (with one CTA per head block of the group)
+// walks its range, which may span several units.  Each maximal piece of a
+// unit inside a range produces one normalised partial output and its LSE
+// in slot (range + unit) of the workspace; the combine kernel merges the
+// pieces of each unit in range order.  Every SM gets the same number of
+// key tiles whatever the mix of sequence lengths.
 //
 // MLA absorbed mode ("Full 路线" sections 4.2-4.3): K rows are the cached
 // [c_kv | k_pe] rows (d_k = 576) and V is the first 512 columns of the same
 // rows (d_v = 512), read through a second tensor map over the same memory.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
-// and issues UMMA, warps 2-5 run the softmax (thread = key row of the tile;
-// for O^T, thread = d_v row of each 128-row block) and the epilogue.
+// Warp roles (192 threads): warp 0 lane 0 streams K/V chunks through the
+// ring and lane 1 loads Q^T per piece (both TMA), warp 1 allocates TMEM and
+// issues UMMA, warps 2-5 run the softmax (thread = key row of the tile; for
+// O^T, thread = d_v row of each 128-row block) and the epilogues.
 #pragma once
 
 #include "sm100.cuh"
@@ -30,13 +39,11 @@
 namespace attn {
 
 struct DecodeParams {
-  const void* q;         // [B, Hq, 1, d_k]
-  int64_t q_sb, q_sh;    // element strides of q
   const int32_t* skv;    // [B] keys per sequence (device)
-  float* ws_o;           // [B, Hq, num_splits, d_v] normalised partial outputs
-  float* ws_lse;         // [B, Hq, num_splits] partial LSE (natural log)
+  float* ws_o;           // [ranges + B*Hkv][G][d_v] normalised partial outputs
+  float* ws_lse;         // [ranges + B*Hkv][G] partial LSE (natural log)
   int B, Hq, Hkv, G;
-  int num_splits, split_tiles, head_blocks;
+  int ranges, head_blocks;
   float scale_log2;      // scale * log2(e)
   uint64_t timeout_ns;
 };
@@ -47,6 +54,8 @@ constexpr uint32_t ceil_pow2_cols(uint32_t n) {
   return c;
 }
 
+__device__ __forceinline__ int key_tiles(int skv) { return (skv + 127) >> 7; }
+
 template <int DK, int DV, int NH>
 struct DecodeTraits {
   static constexpr int TILE = 128;                 // keys per tile (MMA M)
@@ -54,37 +63,117 @@ struct DecodeTraits {
   static constexpr int KSLOTS = (KCH + 1) & ~1;    // ring slots per tile's K (even)
   static constexpr int VCH = DV / 64;              // 64-column V chunks per tile
   static constexpr int DVB = DV / 128;             // 128-row blocks of O^T
-  static constexpr int RING = (DK == 576) ? 6 : (DK == 512 ? 4 : 6);
-  static constexpr int MIN_CTAS = (DK == 576) ? 1 : 2;
+  static constexpr int CTAS = (DK == 128) ? 2 : 1; // resident CTAs per SM
+  static constexpr int RING = (DK == 576) ? 8 : (DK == 512 ? 12 : 6);
+  static constexpr int NPT = (DK == 576) ? 1 : 2;  // P^T buffers
   static constexpr int SLOT = 16384;               // one [128 x 64] 2-byte chunk
   static constexpr int QT_CHUNK = NH * 128;        // one [NH x 64] chunk of Q^T
   static constexpr int PT_BYTES = NH * TILE * 2;   // one P^T buffer
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_QT = OFF_RING + RING * SLOT;
   static constexpr int OFF_PT = OFF_QT + KCH * QT_CHUNK;
-  static constexpr int OFF_RED = OFF_PT + 2 * PT_BYTES;         // float [2][4][NH]
+  static constexpr int OFF_RED = OFF_PT + NPT * PT_BYTES;       // float [2][4][NH]
   static constexpr int OFF_M = OFF_RED + 2 * 4 * NH * 4;        // float [NH] running max
   static constexpr int OFF_ALPHA = OFF_M + NH * 4;              // float [NH] rescale factors
   static constexpr int OFF_L = OFF_ALPHA + NH * 4;              // float [NH] final sums
-  static constexpr int OFF_FLAGS = OFF_L + NH * 4;              // int [4]: any[2], abort, tmem
+  static constexpr int OFF_SCAN = OFF_L + NH * 4;               // int64 [8] block scan
+  static constexpr int OFF_SCHED = OFF_SCAN + 64;               // int [4] range start
+  static constexpr int OFF_FLAGS = OFF_SCHED + 16;              // int [4]: any[2], abort, tmem
   static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
-  // barriers: full[RING], empty[RING], s_full[2], s_free[2], p_full[2], o_done[2], q_full,
+  // full[RING], empty[RING], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full, q_free,
   // red_full[2], stat_ready[2], drain
-  static constexpr int NBAR = 2 * RING + 14;
+  static constexpr int NBAR = 2 * RING + 11 + 2 * NPT;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;  // + alignment slack
   static constexpr int TMEM_S = 0;                  // S^T double buffer: 2 x NH columns
   static constexpr int TMEM_O = 2 * NH;             // O^T: DVB x NH columns
   static constexpr uint32_t TMEM_COLS = ceil_pow2_cols(2 * NH + DVB * NH);
   static_assert(KCH * QT_CHUNK % 1024 == 0, "Q^T chunks must keep 1024-byte alignment");
+  static_assert(OFF_PT % 1024 == 0, "P^T alignment");
   static_assert(RING % 2 == 0 && KSLOTS % 2 == 0 && VCH % 2 == 0, "V chunk pairs need even slots");
   static_assert(NH % 16 == 0 && NH <= 256, "MMA N");
-  static_assert(TMEM_COLS <= 512, "TMEM");
-  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(TMEM_COLS * CTAS <= 512, "TMEM");
+  static_assert(SMEM_BYTES * CTAS <= 232448, "shared memory");
 };
 
+// Walks the pieces of one key range: consecutive (sequence b, kv head) units
+// in b-major order, each piece covering tiles [tile0, tile0 + ntiles) of one
+// unit.  Every role of the CTA runs its own copy over the same range.
+struct PieceWalker {
+  const int32_t* skv;
+  int B, Hkv;
+  int b, kvh, off, remaining;
+
+  __device__ bool next(int& pb, int& pkvh, int& tile0, int& ntiles) {
+    if (remaining <= 0) return false;
+    const int tb = key_tiles(skv[b]);
+    const int n = min(remaining, tb - off);
+    pb = b;
+    pkvh = kvh;
+    tile0 = off;
+    ntiles = n;
+    remaining -= n;
+    off = 0;
+    if (remaining > 0) {
+      if (++kvh == Hkv) {
+        kvh = 0;
+        do { ++b; } while (b < B && key_tiles(skv[b]) == 0);
+      }
+    }
+    return true;
+  }
+};
+
+// Range `r` of min(R, T) equal ranges over the T concatenated key tiles of
+// all units (unit u = b * Hkv + kvh holds ceil(skv[b] / 128) tiles).  Called
+// by all threads of the CTA; leaves the range's first unit, tile offset and
+// length in sched[0..3] (length 0: no range r).
+__device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv, int R, int r,
+                                             long long* scan, int* sched) {
+  const int tid = threadIdx.x;
+  const int nt = blockDim.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int c = (B + nt - 1) / nt;
+  const int lo = min(B, tid * c), hi = min(B, lo + c);
+  long long mine = 0;
+  for (int b = lo; b < hi; ++b) mine += key_tiles(skv[b]);
+  long long v = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) scan[warp] = v;
+  __syncthreads();
+  long long before = 0, total = 0;
+  for (int w = 0; w < (nt >> 5); ++w) {
+    if (w < warp) before += scan[w];
+    total += scan[w];
+  }
+  const long long T = total * Hkv;
+  // With fewer tiles than ranges only the first T ranges are used, so that
+  // every range in use holds at least one tile (the combine relies on it).
+  const long long Re = T < R ? T : R;
+  const long long x0 = r < Re ? (long long)r * T / Re : T;
+  const long long x1 = r < Re ? (long long)(r + 1) * T / Re : T;
+  if (tid == 0) sched[3] = (int)(x1 - x0);
+  long long run = before + v - mine;  // tiles of sequences before `lo`
+  for (int b = lo; b < hi; ++b) {
+    const int tb = key_tiles(skv[b]);
+    const long long base = run * Hkv;
+    if (tb > 0 && x0 < x1 && x0 >= base && x0 < base + (long long)tb * Hkv) {
+      sched[0] = b;
+      sched[1] = (int)((x0 - base) / tb);
+      sched[2] = (int)((x0 - base) % tb);
+    }
+    run += tb;
+  }
+  __syncthreads();
+}
+
 template <int DK, int DV, int NH, bool BF16>
-__global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
-    decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using T = DecodeTraits<DK, DV, NH>;
   extern __shared__ uint8_t smem_raw[];
@@ -92,16 +181,8 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
 
-  const int hb = blockIdx.x % p.head_blocks;
-  const int split = blockIdx.x / p.head_blocks;
-  const int b = blockIdx.y;
-  const int kvh = blockIdx.z;
-  const int skv = p.skv[b];
-  const int tok_begin = split * p.split_tiles * T::TILE;
-  if (tok_begin >= skv) return;  // nothing of this sequence in this split (uniform)
-  const int tok_end = min(skv, tok_begin + p.split_tiles * T::TILE);
-  const int ntiles = (tok_end - tok_begin + T::TILE - 1) / T::TILE;
-  const int h0 = kvh * p.G + hb * NH;            // first query head of this CTA
+  const int hb = blockIdx.x % p.head_blocks;     // head block of the group
+  const int rng = blockIdx.x / p.head_blocks;    // key range
   const int nvalid = min(NH, p.G - hb * NH);     // real heads among the NH rows
 
   const uint32_t ring = sbase + T::OFF_RING;
@@ -111,6 +192,8 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
   float* m_sm = reinterpret_cast<float*>(smem + T::OFF_M);
   float* alpha_sm = reinterpret_cast<float*>(smem + T::OFF_ALPHA);
   float* l_sm = reinterpret_cast<float*>(smem + T::OFF_L);
+  long long* scan = reinterpret_cast<long long*>(smem + T::OFF_SCAN);
+  int* sched = reinterpret_cast<int*>(smem + T::OFF_SCHED);
   volatile int* flags = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
   volatile int* abort_flag = flags + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 12);
@@ -119,10 +202,11 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
   auto empty_bar = [&](int s) { return bar0 + 8u * (T::RING + s); };
   const uint32_t s_full = bar0 + 8u * (2 * T::RING);      // [2]
   const uint32_t s_free = s_full + 16;                    // [2]
-  const uint32_t p_full = s_free + 16;                    // [2]
-  const uint32_t o_done = p_full + 16;                    // [2]
-  const uint32_t q_full = o_done + 16;
-  const uint32_t red_full = q_full + 8;                   // [2]
+  const uint32_t p_full = s_free + 16;                    // [NPT]
+  const uint32_t o_done = p_full + 8 * T::NPT;            // [NPT]
+  const uint32_t q_full = o_done + 8 * T::NPT;
+  const uint32_t q_free = q_full + 8;
+  const uint32_t red_full = q_free + 8;                   // [2]
   const uint32_t stat_ready = red_full + 16;              // [2]
   const uint32_t drain = stat_ready + 16;
 
@@ -137,14 +221,15 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
       mbar_init(s_free + 8 * i, 128);
-      mbar_init(p_full + 8 * i, 128);
-      mbar_init(o_done + 8 * i, 1);
-    }
-    mbar_init(q_full, 128);
-    for (int i = 0; i < 2; ++i) {
       mbar_init(red_full + 8 * i, 128);
       mbar_init(stat_ready + 8 * i, NH);
     }
+    for (int i = 0; i < T::NPT; ++i) {
+      mbar_init(p_full + 8 * i, 128);
+      mbar_init(o_done + 8 * i, 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     mbar_init(drain, 1);
     flags[0] = 0;
     flags[1] = 0;
@@ -155,26 +240,39 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
+  locate_range(p.skv, p.B, p.Hkv, p.ranges, rng, scan, sched);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int count = sched[3];
+  auto walker = [&]() {
+    PieceWalker w;
+    w.skv = p.skv;
+    w.B = p.B;
+    w.Hkv = p.Hkv;
+    w.b = sched[0];
+    w.kvh = sched[1];
+    w.off = sched[2];
+    w.remaining = count;
+    return w;
+  };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (count > 0) {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ producer: K/V ring
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const uint64_t pol = l2_policy_evict_first();
       int slot = 0;
       uint32_t ph = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* map, int c0, int c1) {
+      auto load = [&](const CUtensorMap* map, int c0, int tok, int kvh, int b) {
         if (!ok) return;
         ok = mbar_wait(empty_bar(slot), ph ^ 1u, abort_flag, p.timeout_ns, 1);
         if (!ok) return;
         mbar_arrive_expect_tx(full_bar(slot), T::SLOT);
-        tma_load_4d(ring + slot * T::SLOT, map, full_bar(slot), c0, c1, kvh, b, pol);
+        tma_load_4d(ring + slot * T::SLOT, map, full_bar(slot), c0, tok, kvh, b, pol);
         if (++slot == T::RING) { slot = 0; ph ^= 1u; }
       };
       auto phantom = [&]() {
@@ -184,37 +282,59 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
         mbar_arrive(full_bar(slot));
         if (++slot == T::RING) { slot = 0; ph ^= 1u; }
       };
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int t0 = tok_begin + j * T::TILE;
-        for (int c = 0; c < T::KCH; ++c) load(&tmK, c * 64, t0);
-        if (T::KSLOTS > T::KCH) phantom();
-        if (j >= 1)
-          for (int c = 0; c < T::VCH; ++c) load(&tmV, c * 64, t0 - T::TILE);
+      PieceWalker w = walker();
+      int b, kvh, t0, n;
+      int pv_tok = -1, pv_kvh = 0, pv_b = 0;  // tile whose V is still to be loaded
+      auto load_v = [&]() {
+        for (int c = 0; c < T::VCH; ++c) load(&tmV, c * 64, pv_tok, pv_kvh, pv_b);
+      };
+      while (ok && w.next(b, kvh, t0, n)) {
+        for (int i = 0; i < n && ok; ++i) {
+          const int tok = (t0 + i) * T::TILE;
+          if (i == 0 && pv_tok >= 0) load_v();  // finish the previous piece first
+          for (int c = 0; c < T::KCH; ++c) load(&tmK, c * 64, tok, kvh, b);
+          if (T::KSLOTS > T::KCH) phantom();
+          if (i > 0) load_v();
+          pv_tok = tok;
+          pv_kvh = kvh;
+          pv_b = b;
+        }
       }
-      {
-        const int t0 = tok_begin + (ntiles - 1) * T::TILE;
-        for (int c = 0; c < T::VCH; ++c) load(&tmV, c * 64, t0);
+      if (pv_tok >= 0) load_v();
+      if (!ok) {  // give issued copies time to land before the CTA leaves
+        const uint64_t t0n = global_timer_ns();
+        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
       }
-      // On abort, give every copy this thread started time to land before
-      // the CTA leaves (a tile copy takes microseconds; wait 2 ms).
+    } else if (warp == 0 && lane == 1) {
+      // ------------------------------------------------ producer: Q^T per piece
+      tma_prefetch_desc(&tmQ);
+      const uint64_t pol = l2_policy_evict_first();
+      PieceWalker w = walker();
+      int b, kvh, t0, n, k = 0;
+      bool ok = true;
+      while (ok && w.next(b, kvh, t0, n)) {
+        if (k > 0) ok = mbar_wait(q_free, (k - 1) & 1, abort_flag, p.timeout_ns, 3);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, T::KCH * T::QT_CHUNK);
+        for (int c = 0; c < T::KCH; ++c)
+          tma_load_3d(qt + c * T::QT_CHUNK, &tmQ, q_full, c * 64, kvh * p.G + hb * NH, b, pol);
+        ++k;
+      }
       if (!ok) {
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+        const uint64_t t0n = global_timer_ns();
+        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------ MMA issuer
       constexpr uint32_t idS = umma_idesc(128, NH, BF16, false, false);
       constexpr uint32_t idO = umma_idesc(128, NH, BF16, true, true);
       int slot = 0;
       uint32_t ph = 0;
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.timeout_ns, 3);
-      tc_fence_after();
-      auto pv = [&](int t) {
+      bool ok = true;
+      auto pv = [&](int t, bool first_of_piece) {
         if (!ok) return;
-        const int pb = t & 1;
-        ok = mbar_wait(p_full + 8 * pb, (t >> 1) & 1, abort_flag, p.timeout_ns, 4);
+        const int pb = t % T::NPT;
+        ok = mbar_wait(p_full + 8 * pb, (t / T::NPT) & 1, abort_flag, p.timeout_ns, 4);
         if (!ok) return;
         tc_fence_after();
         const uint32_t bbase = pt + pb * T::PT_BYTES;
@@ -233,7 +353,7 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
             // B = P^T: MN-major, no swizzle; 8x8 core matrices, 8-head groups
             // 128 bytes apart (SBO), 8-key groups NH*16 bytes apart (LBO).
             const uint64_t bd = umma_sdesc(bbase + ks * 2 * NH * 16, NH * 16, 128, SMEM_NOSWIZZLE);
-            umma_ss(tmem + T::TMEM_O + i * NH, ad, bd, idO, (t > 0 || ks > 0) ? 1u : 0u);
+            umma_ss(tmem + T::TMEM_O + i * NH, ad, bd, idO, (!first_of_piece || ks > 0) ? 1u : 0u);
           }
           umma_commit(empty_bar(slot));
           umma_commit(empty_bar(slot + 1));
@@ -242,242 +362,246 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
         }
         umma_commit(o_done + 8 * pb);
       };
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int sb = j & 1;
-        if (j >= 2) ok = mbar_wait(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 6);
-        if (!ok) break;
-        tc_fence_after();
-        for (int c = 0; c < T::KCH && ok; ++c) {
-          ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 7);
+      PieceWalker w = walker();
+      int b, kvh, t0, n, j = 0, k = 0;
+      bool prev_first = false;
+      while (ok && w.next(b, kvh, t0, n)) {
+        for (int i = 0; i < n && ok; ++i, ++j) {
+          const int sb = j & 1;
+          if (i == 0 && j > 0) pv(j - 1, prev_first);  // finish the previous piece first
+          if (i == 0) {
+            ok = ok && mbar_wait(q_full, k & 1, abort_flag, p.timeout_ns, 6);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (j >= 2) ok = mbar_wait(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 7);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t abase = ring + slot * T::SLOT;
-          const uint32_t bbase = qt + c * T::QT_CHUNK;
+          for (int c = 0; c < T::KCH && ok; ++c) {
+            ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 8);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t abase = ring + slot * T::SLOT;
+            const uint32_t bbase = qt + c * T::QT_CHUNK;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
-            // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
-            const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
-            const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
-            umma_ss(tmem + T::TMEM_S + sb * NH, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(empty_bar(slot));
-          if (++slot == T::RING) { slot = 0; ph ^= 1u; }
-        }
-        if (ok && T::KSLOTS > T::KCH) {
-          ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 8);
-          if (ok) {
-            mbar_arrive(empty_bar(slot));
+            for (int ks = 0; ks < 4; ++ks) {
+              // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
+              // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
+              const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
+              const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
+              umma_ss(tmem + T::TMEM_S + sb * NH, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(empty_bar(slot));
             if (++slot == T::RING) { slot = 0; ph ^= 1u; }
           }
+          if (ok && T::KSLOTS > T::KCH) {
+            ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 9);
+            if (ok) {
+              mbar_arrive(empty_bar(slot));
+              if (++slot == T::RING) { slot = 0; ph ^= 1u; }
+            }
+          }
+          if (!ok) break;
+          umma_commit(s_full + 8 * sb);
+          if (i == n - 1) umma_commit(q_free);  // Q^T of this piece no longer read
+          if (i > 0) pv(j - 1, prev_first);
+          prev_first = (i == 0);
         }
-        if (!ok) break;
-        umma_commit(s_full + 8 * sb);
-        if (j >= 1) pv(j - 1);
+        ++k;
       }
-      pv(ntiles - 1);
+      if (ok && j > 0) pv(j - 1, prev_first);
       if (!ok) {
         // Gave up: let every MMA already issued finish before TMEM is freed.
         umma_commit(drain);
         volatile int never = 0;
-        mbar_wait(drain, 0, &never, 1000000ull, 13);
+        mbar_wait(drain, 0, &never, 1000000ull, 10);
       }
-    }
-  } else {
-    // ------------------------------------------------------------ softmax
-    // Cross-warp exchanges use mbarriers with bounded waits (red_full: all
-    // 128 partial maxima written; stat_ready: the per-head maxima, rescale
-    // factors and the "any head rescaled" flag published), so that a wait
-    // that gives up can never leave the other warps parked on a barrier.
-    // These threads do not consult the abort flag: all 128 wait on the same
-    // barriers, so they either all see a barrier complete or all time out.
-    const int st = threadIdx.x - 64;       // 0..127
-    const int wq = warp & 3;               // TMEM lane quarter of this warp
-    const int row = wq * 32 + lane;        // key row of S^T / d_v row of O^T blocks
-    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    volatile int own_abort = 0;
-    auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
-      return mbar_wait(bar, parity, &own_abort, p.timeout_ns, id);
-    };
-
-    // Q^T -> shared memory, K-major 128-byte-swizzled [NH x 64] chunks;
-    // rows past the group's heads are zero.
-    {
-      const uint8_t* qg = reinterpret_cast<const uint8_t*>(p.q);
-      constexpr int PIECES_PER_ROW = DK / 8;  // 16-byte pieces
-      for (int idx = st; idx < NH * PIECES_PER_ROW; idx += 128) {
-        const int r = idx / PIECES_PER_ROW;
-        const int col = (idx % PIECES_PER_ROW) * 8;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nvalid) {
-          const int64_t off = (int64_t)b * p.q_sb + (int64_t)(h0 + r) * p.q_sh + col;
-          val = __ldg(reinterpret_cast<const uint4*>(qg + off * 2));
-        }
-        st_shared_v4(qt + (col / 64) * T::QT_CHUNK + sw128_offset(r, col % 64), val.x, val.y,
-                     val.z, val.w);
-      }
+    } else if (warp >= 2) {
+      // ------------------------------------------------ softmax + epilogues
+      // Cross-warp exchanges use mbarriers with bounded waits (red_full: all
+      // 128 partial values written; stat_ready: per-head statistics
+      // published), so a wait that gives up can never strand the other warps
+      // on a barrier.  These threads ignore the abort flag: all 128 wait on
+      // the same barriers, so they either all see one complete or all time out.
+      const int st = threadIdx.x - 64;       // 0..127
+      const int wq = warp & 3;               // TMEM lane quarter of this warp
+      const int row = wq * 32 + lane;        // key row of S^T / d_v row of O^T blocks
+      const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+      volatile int own_abort = 0;
+      auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
+        return mbar_wait(bar, parity, &own_abort, p.timeout_ns, id);
+      };
       if (st < NH) m_sm[st] = -INFINITY;
-      fence_proxy_async_smem();
-      mbar_arrive(q_full);
-      named_bar_sync(1, 128);  // m_sm initialised before anyone reads it
-    }
+      named_bar_sync(1, 128);
 
-    float l[NH];
+      PieceWalker w = walker();
+      int b, kvh, t0, n, j = 0, r = 0;
+      bool ok = true;
+      while (ok && w.next(b, kvh, t0, n)) {
+        const int skv_b = p.skv[b];
+        const int64_t slot_id = (int64_t)rng + (int64_t)b * p.Hkv + kvh;  // workspace slot
+        float l[NH];
 #pragma unroll
-    for (int h = 0; h < NH; ++h) l[h] = 0.f;
-    bool ok = true;
+        for (int h = 0; h < NH; ++h) l[h] = 0.f;
 
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int sb = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      ok = wait(s_full + 8 * sb, par, 9);
-      if (!ok) break;
-      tc_fence_after();
-      float s[NH];
-#pragma unroll
-      for (int g = 0; g < NH / 16; ++g) {
-        float tmp[16];
-        tmem_ld16(tmem + lane_base + T::TMEM_S + sb * NH + g * 16, tmp);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) s[g * 16 + i] = tmp[i];
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free + 8 * sb);
-
-      // per-head maximum over the tile's 128 keys
-      const bool valid = tok_begin + j * T::TILE + row < tok_end;
-      float* rbuf = red + sb * 4 * NH;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float v = valid ? s[h] * p.scale_log2 : -INFINITY;
-        s[h] = v;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) rbuf[wq * NH + h] = v;
-      }
-      mbar_arrive(red_full + 8 * sb);
-      ok = wait(red_full + 8 * sb, par, 14);
-      if (!ok) break;
-      if (st == 0) flags[sb ^ 1] = 0;
-      if (st < NH) {
-        const float tm = fmaxf(fmaxf(rbuf[st], rbuf[NH + st]), fmaxf(rbuf[2 * NH + st], rbuf[3 * NH + st]));
-        const float mo = m_sm[st];
-        // Keep the stale maximum unless the tile's exceeds it by more than
-        // 8 (log2 units): exp2(s - m) then stays <= 256, and the final
-        // division by the sum accumulated against the same maximum is exact.
-        const bool need = tm > mo + 8.f;
-        const float mn = need ? tm : mo;
-        alpha_sm[st] = need ? ex2(mo - mn) : 1.f;
-        m_sm[st] = mn;
-        if (need) flags[sb] = 1;
-        mbar_arrive(stat_ready + 8 * sb);
-      }
-      ok = wait(stat_ready + 8 * sb, par, 15);
-      if (!ok) break;
-      const bool any = flags[sb] != 0;
-
-      if (j >= 2) {  // P^T buffer sb was last read by PV(j-2)
-        ok = wait(o_done + 8 * sb, ((j - 2) >> 1) & 1, 10);
-        if (!ok) break;
-      }
-      if (any && j >= 1) {  // rescale O^T once PV(j-1) has landed
-        ok = wait(o_done + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, 11);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int i = 0; i < T::DVB; ++i) {
+        for (int i = 0; i < n && ok; ++i, ++j, ++r) {
+          const int sb = j & 1;
+          const int rb = r & 1;
+          const uint32_t rpar = (r >> 1) & 1;
+          ok = wait(s_full + 8 * sb, (j >> 1) & 1, 11);
+          if (!ok) break;
+          tc_fence_after();
+          float s[NH];
 #pragma unroll
           for (int g = 0; g < NH / 16; ++g) {
-            float o[16];
-            const uint32_t ta = tmem + lane_base + T::TMEM_O + i * NH + g * 16;
-            tmem_ld16(ta, o);
-            tmem_wait_ld();
+            float tmp[16];
+            tmem_ld16(tmem + lane_base + T::TMEM_S + sb * NH + g * 16, tmp);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] *= alpha_sm[g * 16 + c];
-            tmem_st16(ta, o);
+            for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
           }
-        }
-        tmem_wait_st();
-      }
-#pragma unroll
-      for (int h = 0; h < NH; ++h) l[h] *= alpha_sm[h];
-
-      // P^T row for this key: NH values, written as MN-major core matrices.
-      const uint32_t prow = pt + sb * T::PT_BYTES + (row >> 3) * (NH * 16) + (row & 7) * 16;
-#pragma unroll
-      for (int g = 0; g < NH / 8; ++g) {
-        uint32_t u[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int h = g * 8 + 2 * e;
-          const float p0 = s[h] == -INFINITY ? 0.f : ex2(s[h] - m_sm[h]);
-          const float p1 = s[h + 1] == -INFINITY ? 0.f : ex2(s[h + 1] - m_sm[h + 1]);
-          u[e] = pack2(p0, p1, BF16);
-          l[h] += p0;
-          l[h + 1] += p1;
-        }
-        st_shared_v4(prow + g * 128, u[0], u[1], u[2], u[3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full + 8 * sb);
-    }
-
-    // ---------------------------------------------------------- epilogue
-    if (ok) {
-      const int last = ntiles - 1;
-      ok = wait(o_done + 8 * (last & 1), (last >> 1) & 1, 12);
-    }
-    if (ok) {
-      tc_fence_after();
-      // the reduction buffers and barriers continue their per-tile sequence
-      const int sb = ntiles & 1;
-      const uint32_t par = (ntiles >> 1) & 1;
-      float* rbuf = red + sb * 4 * NH;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        float v = l[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) rbuf[wq * NH + h] = v;
-      }
-      mbar_arrive(red_full + 8 * sb);
-      ok = wait(red_full + 8 * sb, par, 16);
-      if (ok && st < NH) {
-        const float L = (rbuf[st] + rbuf[NH + st]) + (rbuf[2 * NH + st] + rbuf[3 * NH + st]);
-        l_sm[st] = L;
-        if (st < nvalid) {
-          const int64_t idx = ((int64_t)b * p.Hq + h0 + st) * p.num_splits + split;
-          p.ws_lse[idx] = L > 0.f ? (m_sm[st] + __log2f(L)) * 0.69314718055994531f : -INFINITY;
-        }
-        mbar_arrive(stat_ready + 8 * sb);
-      }
-      if (ok) ok = wait(stat_ready + 8 * sb, par, 17);
-    }
-    if (ok) {
-#pragma unroll 1
-      for (int i = 0; i < T::DVB; ++i) {
-#pragma unroll
-        for (int g = 0; g < NH / 16; ++g) {
-          float o[16];
-          tmem_ld16(tmem + lane_base + T::TMEM_O + i * NH + g * 16, o);
           tmem_wait_ld();
-          const int d = i * 128 + row;
+          tc_fence_before();
+          mbar_arrive(s_free + 8 * sb);
+
+          // per-head maximum over the tile's 128 keys
+          const bool valid = (t0 + i) * T::TILE + row < skv_b;
+          float* rbuf = red + rb * 4 * NH;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int h = g * 16 + c;
-            if (h < nvalid) {
-              const float L = l_sm[h];
-              const int64_t idx = (((int64_t)b * p.Hq + h0 + h) * p.num_splits + split) * DV + d;
-              p.ws_o[idx] = L > 0.f ? o[c] / L : 0.f;
+          for (int h = 0; h < NH; ++h) {
+            float v = valid ? s[h] * p.scale_log2 : -INFINITY;
+            s[h] = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) rbuf[wq * NH + h] = v;
+          }
+          mbar_arrive(red_full + 8 * rb);
+          ok = wait(red_full + 8 * rb, rpar, 12);
+          if (!ok) break;
+          if (st == 0) flags[rb ^ 1] = 0;
+          if (st < NH) {
+            const float tm =
+                fmaxf(fmaxf(rbuf[st], rbuf[NH + st]), fmaxf(rbuf[2 * NH + st], rbuf[3 * NH + st]));
+            const float mo = m_sm[st];
+            // Keep the stale maximum unless the tile's exceeds it by more than
+            // 8 (log2 units): exp2(s - m) then stays <= 256, and the final
+            // division by the sum accumulated against the same maximum is exact.
+            const bool need = tm > mo + 8.f;
+            const float mn = need ? tm : mo;
+            alpha_sm[st] = need ? ex2(mo - mn) : 1.f;
+            m_sm[st] = mn;
+            if (need) flags[rb] = 1;
+            mbar_arrive(stat_ready + 8 * rb);
+          }
+          ok = wait(stat_ready + 8 * rb, rpar, 13);
+          if (!ok) break;
+          const bool any = flags[rb] != 0;
+
+          const int pb = j % T::NPT;
+          if (j >= T::NPT) {  // P^T buffer pb was last read by PV(j - NPT)
+            ok = wait(o_done + 8 * pb, ((j - T::NPT) / T::NPT) & 1, 14);
+            if (!ok) break;
+          }
+          if (any && i > 0) {  // rescale O^T once PV(j-1) has landed
+            ok = wait(o_done + 8 * ((j - 1) % T::NPT), ((j - 1) / T::NPT) & 1, 15);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int d = 0; d < T::DVB; ++d) {
+#pragma unroll
+              for (int g = 0; g < NH / 16; ++g) {
+                float o[16];
+                const uint32_t ta = tmem + lane_base + T::TMEM_O + d * NH + g * 16;
+                tmem_ld16(ta, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) o[c] *= alpha_sm[g * 16 + c];
+                tmem_st16(ta, o);
+              }
+            }
+            tmem_wait_st();
+          }
+#pragma unroll
+          for (int h = 0; h < NH; ++h) l[h] *= alpha_sm[h];
+
+          // P^T row for this key: NH values, written as MN-major core matrices.
+          const uint32_t prow = pt + pb * T::PT_BYTES + (row >> 3) * (NH * 16) + (row & 7) * 16;
+#pragma unroll
+          for (int g = 0; g < NH / 8; ++g) {
+            uint32_t u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int h = g * 8 + 2 * e;
+              const float p0 = s[h] == -INFINITY ? 0.f : ex2(s[h] - m_sm[h]);
+              const float p1 = s[h + 1] == -INFINITY ? 0.f : ex2(s[h + 1] - m_sm[h + 1]);
+              u[e] = pack2(p0, p1, BF16);
+              l[h] += p0;
+              l[h + 1] += p1;
+            }
+            st_shared_v4(prow + g * 128, u[0], u[1], u[2], u[3]);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(p_full + 8 * pb);
+        }
+        if (!ok) break;
+
+        // ---------------------------------------------- epilogue of the piece
+        {
+          const int t = j - 1;  // last tile of the piece
+          ok = wait(o_done + 8 * (t % T::NPT), (t / T::NPT) & 1, 16);
+          if (!ok) break;
+          tc_fence_after();
+          const int rb = r & 1;
+          const uint32_t rpar = (r >> 1) & 1;
+          float* rbuf = red + rb * 4 * NH;
+#pragma unroll
+          for (int h = 0; h < NH; ++h) {
+            float v = l[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) rbuf[wq * NH + h] = v;
+          }
+          mbar_arrive(red_full + 8 * rb);
+          ok = wait(red_full + 8 * rb, rpar, 17);
+          if (!ok) break;
+          if (st == 0) flags[rb ^ 1] = 0;
+          if (st < NH) {
+            const float L = (rbuf[st] + rbuf[NH + st]) + (rbuf[2 * NH + st] + rbuf[3 * NH + st]);
+            l_sm[st] = L;
+            if (st < nvalid)
+              p.ws_lse[slot_id * p.G + hb * NH + st] =
+                  L > 0.f ? (m_sm[st] + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+            m_sm[st] = -INFINITY;  // the next piece starts afresh
+            mbar_arrive(stat_ready + 8 * rb);
+          }
+          ok = wait(stat_ready + 8 * rb, rpar, 18);
+          if (!ok) break;
+          ++r;
+#pragma unroll 1
+          for (int d = 0; d < T::DVB; ++d) {
+#pragma unroll
+            for (int g = 0; g < NH / 16; ++g) {
+              float o[16];
+              tmem_ld16(tmem + lane_base + T::TMEM_O + d * NH + g * 16, o);
+              tmem_wait_ld();
+              const int dd = d * 128 + row;
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const int h = g * 16 + c;
+                if (h < nvalid) {
+                  const float L = l_sm[h];
+                  p.ws_o[(slot_id * p.G + hb * NH + h) * DV + dd] = L > 0.f ? o[c] / L : 0.f;
+                }
+              }
             }
           }
+          tc_fence_before();
         }
       }
+      if (!ok) *abort_flag = 1;
     }
-    if (!ok) *abort_flag = 1;
   }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -489,9 +613,8 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::MIN_CTAS)
 // ---------------------------------------------------------------- combine
 //
 // out[b,h,0,:] = sum_s exp(lse_s - L) o_s,  L = log sum_s exp(lse_s), over
-// the splits that hold keys of sequence b, in split order (no atomics, so
-// the result is bitwise reproducible: "GQA和MLA详解" section 4 on reduction
-// order).
+// the pieces of unit (b, h / G), in range order (no atomics, so the result
+// is bitwise reproducible: "GQA和MLA详解" section 4 on reduction order).
 struct CombineParams {
   const float* ws_o;
   const float* ws_lse;
@@ -499,40 +622,131 @@ struct CombineParams {
   void* out;
   int64_t o_sb, o_sh;
   float* lse;  // [B, Hq] (Sq == 1) or NULL
-  int B, Hq, DV, num_splits, split_tokens;
+  int B, Hq, Hkv, G, DV, ranges;
 };
+
+// Largest range index r with floor(r * T / R) <= x (the range holding tile x).
+__device__ __forceinline__ long long range_of(long long x, long long T, long long R) {
+  return ((x + 1) * R + T - 1) / T - 1;
+}
 
 template <bool BF16>
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+  // One block per (b, h).  The piece weights w_s = exp(lse_s - L) are
+  // computed once into shared memory; each thread then owns 4 consecutive
+  // d_v columns (float4) of one piece-group g and accumulates its pieces
+  // s = g, g + NG, ... in order; the NG group sums are added in group order.
+  constexpr int MAXS = 1024;
+  __shared__ float w_sm[MAXS];
+  __shared__ float red[4];
+  __shared__ long long redl[8];
+  __shared__ float4 part[128];
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
-  const int skv = p.skv[b];
-  const int n = min(p.num_splits, (skv + p.split_tokens - 1) / p.split_tokens);
-  const float* lse_s = p.ws_lse + (int64_t)bh * p.num_splits;
-  float mx = -INFINITY;
-  for (int s = 0; s < n; ++s) mx = fmaxf(mx, lse_s[s]);
-  float L = -INFINITY;
-  if (n > 0 && mx != -INFINITY) {
-    float acc = 0.f;
-    for (int s = 0; s < n; ++s) acc += __expf(lse_s[s] - mx);
-    L = mx + __logf(acc);
+  const int kvh = h / p.G;
+  const int gh = h % p.G;
+  const int t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
+
+  // tiles of the sequences before b, and of all sequences
+  long long pre = 0, tot = 0;
+  for (int bb = t; bb < p.B; bb += 128) {
+    const int tb = key_tiles(p.skv[bb]);
+    tot += tb;
+    if (bb < b) pre += tb;
   }
-  const float* o_s = p.ws_o + (int64_t)bh * p.num_splits * p.DV;
-  uint8_t* outp = reinterpret_cast<uint8_t*>(p.out) + ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh) * 2;
-  for (int d = threadIdx.x * 2; d < p.DV; d += 256) {
-    float a0 = 0.f, a1 = 0.f;
-    if (L != -INFINITY) {
-      for (int s = 0; s < n; ++s) {
-        const float w = __expf(lse_s[s] - L);
-        const float2 v = *reinterpret_cast<const float2*>(o_s + (int64_t)s * p.DV + d);
-        a0 = fmaf(w, v.x, a0);
-        a1 = fmaf(w, v.y, a1);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  }
+  if (lane == 0) {
+    redl[warp] = pre;
+    redl[4 + warp] = tot;
+  }
+  __syncthreads();
+  pre = (redl[0] + redl[1]) + (redl[2] + redl[3]);
+  tot = (redl[4] + redl[5]) + (redl[6] + redl[7]);
+  const int tu = key_tiles(p.skv[b]);
+  const long long T = tot * p.Hkv;
+  const long long Re = T < p.ranges ? T : p.ranges;  // ranges in use, none empty
+  const long long u = (long long)b * p.Hkv + kvh;
+  int n = 0;
+  long long r_lo = 0;
+  if (tu > 0) {
+    const long long su = pre * p.Hkv + (long long)kvh * tu;
+    r_lo = range_of(su, T, Re);
+    n = (int)(range_of(su + tu - 1, T, Re) - r_lo + 1);
+    n = min(n, MAXS);
+  }
+  // piece s of this unit lives in workspace slot (r_lo + s) + u
+  auto slot = [&](int s) { return (r_lo + s + u) * p.G + gh; };
+
+  float mx = -INFINITY;
+  for (int s = t; s < n; s += 128) mx = fmaxf(mx, p.ws_lse[slot(s)]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float sum = 0.f;
+  if (mx != -INFINITY)
+    for (int s = t; s < n; s += 128) sum += __expf(p.ws_lse[slot(s)] - mx);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  sum = (red[0] + red[1]) + (red[2] + red[3]);
+  const float L = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + __logf(sum);
+  for (int s = t; s < n; s += 128) w_sm[s] = (L == -INFINITY) ? 0.f : __expf(p.ws_lse[slot(s)] - L);
+  __syncthreads();
+
+  const int D4 = p.DV / 4;             // float4 columns (128 or 32)
+  const int NG = 128 / D4;             // piece groups (1 or 4)
+  const int d4 = t % D4;
+  const int g = t / D4;
+  auto src = [&](int s) {
+    return reinterpret_cast<const float4*>(p.ws_o + slot(s) * (long long)p.DV)[d4];
+  };
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = g;
+  for (; s + 3 * NG < n; s += 4 * NG) {  // four independent loads in flight
+    const float4 v0 = src(s), v1 = src(s + NG), v2 = src(s + 2 * NG), v3 = src(s + 3 * NG);
+    const float w0 = w_sm[s], w1 = w_sm[s + NG], w2 = w_sm[s + 2 * NG], w3 = w_sm[s + 3 * NG];
+    acc.x = fmaf(w3, v3.x, fmaf(w2, v2.x, fmaf(w1, v1.x, fmaf(w0, v0.x, acc.x))));
+    acc.y = fmaf(w3, v3.y, fmaf(w2, v2.y, fmaf(w1, v1.y, fmaf(w0, v0.y, acc.y))));
+    acc.z = fmaf(w3, v3.z, fmaf(w2, v2.z, fmaf(w1, v1.z, fmaf(w0, v0.z, acc.z))));
+    acc.w = fmaf(w3, v3.w, fmaf(w2, v2.w, fmaf(w1, v1.w, fmaf(w0, v0.w, acc.w))));
+  }
+  for (; s < n; s += NG) {
+    const float4 v = src(s);
+    const float wv = w_sm[s];
+    acc.x = fmaf(wv, v.x, acc.x);
+    acc.y = fmaf(wv, v.y, acc.y);
+    acc.z = fmaf(wv, v.z, acc.z);
+    acc.w = fmaf(wv, v.w, acc.w);
+  }
+  if (NG > 1) {
+    part[t] = acc;
+    __syncthreads();
+    if (g == 0) {
+      for (int gg = 1; gg < NG; ++gg) {
+        const float4 o = part[gg * D4 + d4];
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
       }
     }
-    *reinterpret_cast<uint32_t*>(outp + (int64_t)d * 2) = pack2(a0, a1, BF16);
   }
-  if (threadIdx.x == 0 && p.lse) p.lse[bh] = L;
+  if (g == 0) {
+    uint8_t* outp =
+        reinterpret_cast<uint8_t*>(p.out) + ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + d4 * 4) * 2;
+    *reinterpret_cast<uint2*>(outp) = make_uint2(pack2(acc.x, acc.y, BF16), pack2(acc.z, acc.w, BF16));
+  }
+  if (t == 0 && p.lse) p.lse[bh] = L;
 }
 
 }  // namespace attn

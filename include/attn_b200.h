@@ -72,9 +72,11 @@ typedef struct {
 typedef struct {
   int path;            /* 0 = prefill kernel, 1 = split-KV decode + combine      */
   int heads_per_cta;   /* decode: query heads packed into one CTA (MMA N)       */
-  int head_blocks;     /* decode: CTAs per (b, kv head) along the query heads   */
-  int num_splits;      /* decode: KV splits per sequence                        */
-  int split_tokens;    /* decode: keys per split (multiple of 128)              */
+  int head_blocks;     /* decode: CTAs per key range along the group's heads    */
+  int kv_ranges;       /* decode: equal ranges the concatenated key tiles of all
+                          (sequence, kv head) pairs are cut into, one persistent
+                          CTA per range and head block                           */
+  int64_t partials;    /* decode: partial-result slots (kv_ranges + B * Hkv)    */
   int dv_parts;        /* prefill: CTAs sharing one q tile, each owning d_v/dv_parts columns */
   int64_t grid_ctas;   /* CTAs of the main kernel                               */
   size_t workspace_bytes;
@@ -92,9 +94,10 @@ attn_status_t attn_plan(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
 
 /*
  * Workspace bytes attn_fwd needs for this problem on the current device
- * (0 for prefill).  Decode stores per-split partial outputs (fp32
- * [B, Hq, splits, d_v]) and partial LSEs (fp32 [B, Hq, splits]) there.
- * Returns 0 for arguments attn_plan rejects.
+ * (0 for prefill).  Decode stores partial outputs (fp32 [partials, G, d_v])
+ * and partial LSEs (fp32 [partials, G]) there, one slot per piece of a
+ * (sequence, kv head) pair that falls in one key range.  Returns 0 for
+ * arguments attn_plan rejects.
  */
 size_t attn_workspace_bytes(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v);
 
@@ -123,10 +126,11 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
  * The two steps attn_fwd enqueues for a decode problem (Sq == 1), callable
  * separately with attn_fwd's arguments (for timing each kernel, or for
  * overlapping the merge with other work):
- *   attn_decode_partial  -- every (sequence, kv head, head block, KV split)
- *                           attends over its keys and writes a normalised
- *                           partial output and its LSE into the workspace;
- *   attn_decode_combine  -- merges the splits of each (b, h) in split order:
+ *   attn_decode_partial  -- one persistent CTA per key range and head block
+ *                           attends over each piece of a (sequence, kv head)
+ *                           pair in its range and writes a normalised partial
+ *                           output and its LSE into the workspace;
+ *   attn_decode_combine  -- merges the pieces of each (b, h) in range order:
  *                           L = ln sum_s exp(lse_s), out = sum_s exp(lse_s - L) o_s
  *                           ("GQA和MLA详解" section 4: a fixed reduction order keeps
  *                           the result bitwise reproducible).

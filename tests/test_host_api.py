@@ -47,12 +47,66 @@ def test_plan_decode_invariants(lib):
         assert pl["path"] == 1
         assert pl["heads_per_cta"] == (64 if dk == 576 else 16)
         assert pl["head_blocks"] == -(-G // pl["heads_per_cta"])
-        assert pl["split_tokens"] % 128 == 0
-        assert pl["num_splits"] * pl["split_tokens"] >= S > (pl["num_splits"] - 1) * pl["split_tokens"]
-        assert pl["grid_ctas"] == B * Hkv * pl["head_blocks"] * pl["num_splits"]
-        n = B * Hq * pl["num_splits"]
+        ctas_per_sm = 2 if dk == 128 else 1
+        assert pl["kv_ranges"] == max(1, 148 * ctas_per_sm // pl["head_blocks"])
+        assert pl["grid_ctas"] == pl["kv_ranges"] * pl["head_blocks"]
+        assert pl["partials"] == pl["kv_ranges"] + B * Hkv
+        n = pl["partials"] * G
         r256 = lambda x: (x + 255) // 256 * 256
         assert pl["workspace_bytes"] == r256(n * dv * 4) + r256(n * 4)
+
+
+def _ranges_pieces(skv, Hkv, R):
+    """Independent model of the decode schedule: concatenated tiles of the
+    (b, kvh) units cut into R equal ranges; pieces = nonempty overlaps."""
+    tiles = [(L + 127) // 128 for L in skv]
+    units = [(b, k, tiles[b]) for b in range(len(skv)) for k in range(Hkv)]
+    T = sum(t for _, _, t in units)
+    R = min(R, T)  # only ranges that hold at least one tile are used
+    bounds = [r * T // R for r in range(R + 1)] if R else [0]
+    pieces, start = [], 0
+    for u, (b, k, t) in enumerate(units):
+        for r in range(R):
+            lo, hi = max(bounds[r], start), min(bounds[r + 1], start + t)
+            if lo < hi:
+                pieces.append((r, u, lo - start, hi - lo))
+        start += t
+    return T, bounds, pieces
+
+
+def test_schedule_slots_unique_and_cover():
+    """Each piece writes workspace slot (range + unit): slots are distinct,
+    stay below kv_ranges + units, and the pieces tile every unit once in
+    range order (what the combine walks)."""
+    import random
+    rnd = random.Random(0)
+    for trial in range(200):
+        B = rnd.randint(1, 40)
+        Hkv = rnd.choice([1, 2, 8])
+        skv = [rnd.choice([0, 1, 127, 128, 129, rnd.randint(0, 9000)]) for _ in range(B)]
+        R = rnd.randint(1, 300)
+        T, bounds, pieces = _ranges_pieces(skv, Hkv, R)
+        slots = [r + u for r, u, _, _ in pieces]
+        assert len(set(slots)) == len(slots)
+        assert all(0 <= s < R + B * Hkv for s in slots)
+        per_unit = {}
+        for r, u, off, n in pieces:
+            per_unit.setdefault(u, []).append((r, off, n))
+        for u, lst in per_unit.items():
+            assert [x[0] for x in lst] == sorted(x[0] for x in lst)
+            pos = 0
+            for r, off, n in lst:
+                assert off == pos
+                pos += n
+            assert pos == (skv[u // Hkv] + 127) // 128
+            # the combine locates the ranges of a unit by this formula
+            t_u = pos
+            s_u = sum((L + 127) // 128 for L in skv[: u // Hkv]) * Hkv + (u % Hkv) * t_u
+            Re = min(R, T)
+            r_of = lambda x: ((x + 1) * Re + T - 1) // T - 1
+            assert r_of(s_u) == lst[0][0] and r_of(s_u + t_u - 1) == lst[-1][0]
+            # every range from the first to the last holds a piece of the unit
+            assert [x[0] for x in lst] == list(range(lst[0][0], lst[-1][0] + 1))
 
 
 def test_plan_prefill(lib):
