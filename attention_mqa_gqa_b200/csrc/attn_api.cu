@@ -98,7 +98,7 @@ bool strides_ok(const attn_strides_t& s) {
 }
 
 // Resident decode CTAs per SM (must match DecodeTraits<...>::CTAS).
-int decode_ctas_per_sm(int d_k) { return d_k == 128 ? 2 : 1; }
+int decode_ctas_per_sm(int d_k) { return d_k == 576 ? 1 : 2; }
 
 bool shape_supported(int Sq, int d_k, int d_v) {
   if (Sq > 1) return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512);
@@ -157,7 +157,7 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
                             const attn_plan_t& pl, cudaStream_t st, int phases) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
-  static_assert(Tr::CTAS == (DK == 128 ? 2 : 1), "decode_ctas_per_sm out of sync");
+  static_assert(Tr::CTAS == (DK == 576 ? 1 : 2), "decode_ctas_per_sm out of sync");
   if (phases & PHASE_PARTIAL) {
     auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
     set_smem(kern, Tr::SMEM_BYTES);

@@ -63,15 +63,17 @@ struct DecodeTraits {
   static constexpr int KSLOTS = (KCH + 1) & ~1;    // ring slots per tile's K (even)
   static constexpr int VCH = DV / 64;              // 64-column V chunks per tile
   static constexpr int DVB = DV / 128;             // 128-row blocks of O^T
-  static constexpr int CTAS = (DK == 128) ? 2 : 1; // resident CTAs per SM
-  static constexpr int RING = (DK == 576) ? 8 : (DK == 512 ? 12 : 6);
+  static constexpr int CTAS = (DK == 576) ? 1 : 2; // resident CTAs per SM
+  static constexpr int RING = (DK == 576) ? 8 : (DK == 512 ? 4 : 6);
   static constexpr int NPT = (DK == 576) ? 1 : 2;  // P^T buffers
+  static constexpr int NQ = (DK == 512) ? 2 : 1;   // Q^T buffers (next piece's Q^T prefetched)
   static constexpr int SLOT = 16384;               // one [128 x 64] 2-byte chunk
   static constexpr int QT_CHUNK = NH * 128;        // one [NH x 64] chunk of Q^T
   static constexpr int PT_BYTES = NH * TILE * 2;   // one P^T buffer
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_QT = OFF_RING + RING * SLOT;
-  static constexpr int OFF_PT = OFF_QT + KCH * QT_CHUNK;
+  static constexpr int QT_BYTES = KCH * QT_CHUNK;   // one Q^T buffer
+  static constexpr int OFF_PT = OFF_QT + NQ * QT_BYTES;
   static constexpr int OFF_RED = OFF_PT + NPT * PT_BYTES;       // float [2][4][NH]
   static constexpr int OFF_M = OFF_RED + 2 * 4 * NH * 4;        // float [NH] running max
   static constexpr int OFF_ALPHA = OFF_M + NH * 4;              // float [NH] rescale factors
@@ -80,20 +82,52 @@ struct DecodeTraits {
   static constexpr int OFF_SCHED = OFF_SCAN + 64;               // int [4] range start
   static constexpr int OFF_FLAGS = OFF_SCHED + 16;              // int [4]: any[2], abort, tmem
   static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
-  // full[RING], empty[RING], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full, q_free,
-  // red_full[2], stat_ready[2], drain
-  static constexpr int NBAR = 2 * RING + 11 + 2 * NPT;
+  // full[RING], empty[RING], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full[NQ],
+  // q_free[NQ], red_full[2], stat_ready[2], drain
+  static constexpr int NBAR = 2 * RING + 9 + 2 * NPT + 2 * NQ;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;  // + alignment slack
   static constexpr int TMEM_S = 0;                  // S^T double buffer: 2 x NH columns
   static constexpr int TMEM_O = 2 * NH;             // O^T: DVB x NH columns
   static constexpr uint32_t TMEM_COLS = ceil_pow2_cols(2 * NH + DVB * NH);
-  static_assert(KCH * QT_CHUNK % 1024 == 0, "Q^T chunks must keep 1024-byte alignment");
+  static_assert(QT_BYTES % 1024 == 0, "Q^T buffers must keep 1024-byte alignment");
   static_assert(OFF_PT % 1024 == 0, "P^T alignment");
   static_assert(RING % 2 == 0 && KSLOTS % 2 == 0 && VCH % 2 == 0, "V chunk pairs need even slots");
   static_assert(NH % 16 == 0 && NH <= 256, "MMA N");
   static_assert(TMEM_COLS * CTAS <= 512, "TMEM");
   static_assert(SMEM_BYTES * CTAS <= 232448, "shared memory");
 };
+
+// Maximum over the 32 lanes of a warp for each of NH values per lane, as a
+// transposed butterfly: at each exchange distance a lane keeps half of its
+// live values (the half its lane bit selects), swaps the other half with
+// its partner and keeps the maxima, so NH/2 + NH/4 + ... shuffles replace
+// 5 * NH.  Afterwards lane l holds in v[0 .. max(NH/32, 1) - 1] the maxima of
+// heads transposed_head<NH>(l, i).
+template <int NH, int N, int OFF>
+__device__ __forceinline__ void transposed_warp_max(float (&v)[NH], int lane) {
+  if constexpr (OFF > 0) {
+    if constexpr (N == 1) {
+      v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], OFF));
+      transposed_warp_max<NH, 1, OFF / 2>(v, lane);
+    } else {
+      constexpr int H = N / 2;
+      const bool upper = (lane & OFF) != 0;
+#pragma unroll
+      for (int i = 0; i < H; ++i) {
+        const float keep = upper ? v[i + H] : v[i];
+        const float send = upper ? v[i] : v[i + H];
+        v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, OFF));
+      }
+      transposed_warp_max<NH, H, OFF / 2>(v, lane);
+    }
+  }
+}
+
+template <int NH>
+__device__ __forceinline__ int transposed_head(int lane, int i) {
+  if constexpr (NH >= 32) return lane * (NH / 32) + i;
+  else return lane / (32 / NH);
+}
 
 // Walks the pieces of one key range: consecutive (sequence b, kv head) units
 // in b-major order, each piece covering tiles [tile0, tile0 + ntiles) of one
@@ -204,9 +238,9 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
   const uint32_t s_free = s_full + 16;                    // [2]
   const uint32_t p_full = s_free + 16;                    // [NPT]
   const uint32_t o_done = p_full + 8 * T::NPT;            // [NPT]
-  const uint32_t q_full = o_done + 8 * T::NPT;
-  const uint32_t q_free = q_full + 8;
-  const uint32_t red_full = q_free + 8;                   // [2]
+  const uint32_t q_full = o_done + 8 * T::NPT;           // [NQ]
+  const uint32_t q_free = q_full + 8 * T::NQ;             // [NQ]
+  const uint32_t red_full = q_free + 8 * T::NQ;           // [2]
   const uint32_t stat_ready = red_full + 16;              // [2]
   const uint32_t drain = stat_ready + 16;
 
@@ -228,8 +262,10 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
       mbar_init(p_full + 8 * i, 128);
       mbar_init(o_done + 8 * i, 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(q_free, 1);
+    for (int i = 0; i < T::NQ; ++i) {
+      mbar_init(q_full + 8 * i, 1);
+      mbar_init(q_free + 8 * i, 1);
+    }
     mbar_init(drain, 1);
     flags[0] = 0;
     flags[1] = 0;
@@ -313,11 +349,14 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
       int b, kvh, t0, n, k = 0;
       bool ok = true;
       while (ok && w.next(b, kvh, t0, n)) {
-        if (k > 0) ok = mbar_wait(q_free, (k - 1) & 1, abort_flag, p.timeout_ns, 3);
+        const int qb = k % T::NQ;
+        if (k >= T::NQ)  // buffer qb was last read by the S^T MMAs of piece k - NQ
+          ok = mbar_wait(q_free + 8 * qb, ((k - T::NQ) / T::NQ) & 1, abort_flag, p.timeout_ns, 3);
         if (!ok) break;
-        mbar_arrive_expect_tx(q_full, T::KCH * T::QT_CHUNK);
+        mbar_arrive_expect_tx(q_full + 8 * qb, T::QT_BYTES);
         for (int c = 0; c < T::KCH; ++c)
-          tma_load_3d(qt + c * T::QT_CHUNK, &tmQ, q_full, c * 64, kvh * p.G + hb * NH, b, pol);
+          tma_load_3d(qt + qb * T::QT_BYTES + c * T::QT_CHUNK, &tmQ, q_full + 8 * qb, c * 64,
+                      kvh * p.G + hb * NH, b, pol);
         ++k;
       }
       if (!ok) {
@@ -370,7 +409,7 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           const int sb = j & 1;
           if (i == 0 && j > 0) pv(j - 1, prev_first);  // finish the previous piece first
           if (i == 0) {
-            ok = ok && mbar_wait(q_full, k & 1, abort_flag, p.timeout_ns, 6);
+            ok = ok && mbar_wait(q_full + 8 * (k % T::NQ), (k / T::NQ) & 1, abort_flag, p.timeout_ns, 6);
             if (!ok) break;
             tc_fence_after();
           }
@@ -382,7 +421,7 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
             if (!ok) break;
             tc_fence_after();
             const uint32_t abase = ring + slot * T::SLOT;
-            const uint32_t bbase = qt + c * T::QT_CHUNK;
+            const uint32_t bbase = qt + (k % T::NQ) * T::QT_BYTES + c * T::QT_CHUNK;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
@@ -403,7 +442,7 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           }
           if (!ok) break;
           umma_commit(s_full + 8 * sb);
-          if (i == n - 1) umma_commit(q_free);  // Q^T of this piece no longer read
+          if (i == n - 1) umma_commit(q_free + 8 * (k % T::NQ));  // this piece's Q^T is free
           if (i > 0) pv(j - 1, prev_first);
           prev_first = (i == 0);
         }
@@ -451,28 +490,32 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           ok = wait(s_full + 8 * sb, (j >> 1) & 1, 11);
           if (!ok) break;
           tc_fence_after();
-          float s[NH];
+          const bool valid = (t0 + i) * T::TILE + row < skv_b;
+          // S^T row of this key (scaled to log2 units, masked), read from TMEM.
+          // It is read twice: once for the maxima and again for the weights,
+          // so that only one NH-wide array is live at a time.
+          auto load_s = [&](float (&x)[NH]) {
 #pragma unroll
-          for (int g = 0; g < NH / 16; ++g) {
-            float tmp[16];
-            tmem_ld16(tmem + lane_base + T::TMEM_S + sb * NH + g * 16, tmp);
+            for (int g = 0; g < NH / 16; ++g) {
+              float tmp[16];
+              tmem_ld16(tmem + lane_base + T::TMEM_S + sb * NH + g * 16, tmp);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
-          }
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(s_free + 8 * sb);
+              for (int e = 0; e < 16; ++e) x[g * 16 + e] = valid ? tmp[e] * p.scale_log2 : -INFINITY;
+            }
+            tmem_wait_ld();
+          };
 
           // per-head maximum over the tile's 128 keys
-          const bool valid = (t0 + i) * T::TILE + row < skv_b;
           float* rbuf = red + rb * 4 * NH;
+          {
+            float v[NH];
+            load_s(v);
+            transposed_warp_max<NH, NH, 16>(v, lane);
+            constexpr int HPL = NH >= 32 ? NH / 32 : 1;
+            if (NH >= 32 || (lane & (32 / NH - 1)) == 0) {
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
-            float v = valid ? s[h] * p.scale_log2 : -INFINITY;
-            s[h] = v;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) rbuf[wq * NH + h] = v;
+              for (int e = 0; e < HPL; ++e) rbuf[wq * NH + transposed_head<NH>(lane, e)] = v[e];
+            }
           }
           mbar_arrive(red_full + 8 * rb);
           ok = wait(red_full + 8 * rb, rpar, 12);
@@ -522,6 +565,11 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           }
 #pragma unroll
           for (int h = 0; h < NH; ++h) l[h] *= alpha_sm[h];
+
+          float s[NH];
+          load_s(s);
+          tc_fence_before();
+          mbar_arrive(s_free + 8 * sb);
 
           // P^T row for this key: NH values, written as MN-major core matrices.
           const uint32_t prow = pt + pb * T::PT_BYTES + (row >> 3) * (NH * 16) + (row & 7) * 16;

@@ -13,9 +13,11 @@ kernel against the measured peaks, the CPU oracle's throughput on a bounded
 sample, and an end-to-end figure through the C ABI with host buffers.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
-and cudaDeviceSynchronize on both sides; CUDA events on the launching stream;
-with N GPUs (torchrun) every rank runs its own replica of the workload and
-the time is the max over ranks.  Inputs are larger than L2 for the decode
+and cudaDeviceSynchronize on both sides, replayed from CUDA graphs that hold
+the steps' C-ABI launches; CUDA events on the replay stream; per-kernel
+durations from external events captured between the kernels.  With N GPUs
+(torchrun) every rank runs its own replica of the workload and the time is
+the max over ranks.  Inputs are larger than L2 for the decode
 workloads (the KV cache alone is 302 MB vs 126 MB L2).
 """
 from __future__ import annotations
@@ -218,36 +220,51 @@ class GpuRunner:
     def launches_per_step(self):
         return 2 if self.decode else 1
 
-    def timed(self, steps, warmup, events_per_kernel=True):
-        """Run warmup + steps; return (total_ms, dominant kernel mean ms,
-        other kernel mean ms)."""
-        for _ in range(warmup):
-            self.call()
+    def _graph(self, nsteps, entry="attn_fwd"):
+        """Capture `nsteps` launches of `entry` (a whole step for attn_fwd)
+        into one CUDA graph on a side stream."""
+        side = torch.cuda.Stream(self.dev)
+        saved, self.stream, self._args = self.stream, side, None
+        graph = torch.cuda.CUDAGraph()
         torch.cuda.synchronize(self.dev)
-        E = lambda: torch.cuda.Event(enable_timing=True)
-        if self.decode and events_per_kernel:
-            ev = [E() for _ in range(2 * steps + 1)]
-            start, end = ev[0], ev[-1]
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for _ in range(nsteps):
+                    self.call(entry)
+        torch.cuda.synchronize(self.dev)
+        self.stream, self._args = saved, None
+        return graph, side
+
+    def _replay_ms(self, graph, side, reps, warmup_reps):
+        with torch.cuda.stream(side):  # replays run on the current stream
+            for _ in range(warmup_reps):
+                graph.replay()
             torch.cuda.synchronize(self.dev)
-            ev[0].record(self.stream)
-            for i in range(steps):
-                self.call("attn_decode_partial")
-                ev[2 * i + 1].record(self.stream)
-                self.call("attn_decode_combine")
-                ev[2 * i + 2].record(self.stream)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(side)
+            for _ in range(reps):
+                graph.replay()
+            b.record(side)
             torch.cuda.synchronize(self.dev)
-            part = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
-            comb = [ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(steps)]
-            return start.elapsed_time(end), statistics.mean(part), statistics.mean(comb)
-        ev = [E() for _ in range(steps + 1)]
-        torch.cuda.synchronize(self.dev)
-        ev[0].record(self.stream)
-        for i in range(steps):
-            self.call()
-            ev[i + 1].record(self.stream)
-        torch.cuda.synchronize(self.dev)
-        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
-        return ev[0].elapsed_time(ev[-1]), statistics.mean(per), 0.0
+        return a.elapsed_time(b)
+
+    def timed(self, steps, warmup):
+        """Warm up, then time exactly `steps` steps replayed from CUDA graphs
+        (captured `per` steps at a time); CUDA events on the replay stream.
+        Returns (total_ms, dominant kernel mean ms, other kernel mean ms).
+        The dominant kernel's duration is timed the same way over graphs of
+        20 back-to-back launches of that kernel alone (for decode the split
+        kernel, whose inputs do not depend on the combine); the combine's is
+        the step time minus that."""
+        per = max(d for d in range(1, min(steps, 20) + 1) if steps % d == 0)
+        graph, side = self._graph(per)
+        total = self._replay_ms(graph, side, steps // per, max(1, warmup // per))
+        del graph
+        if not self.decode:
+            return total, total / steps, 0.0
+        kg, kside = self._graph(20, "attn_decode_partial")
+        k_ms = self._replay_ms(kg, kside, 10, 1) / 200
+        return total, k_ms, max(total / steps - k_ms, 0.0)
 
     def e2e(self, steps, warmup, inp):
         """Same step through the C ABI with the step's inputs in pinned host
@@ -437,9 +454,9 @@ def reference_arm(args, world, rank):
 
 def measure_workload(w, inp, device, steps, warmup, world):
     g = GpuRunner(w, inp, device)
-    if steps is None:  # size the timed region to about 2 s
-        t_ms, _, _ = g.timed(5, 3, events_per_kernel=False)
-        steps = int(min(20000, max(20, 2000.0 / max(t_ms / 5, 1e-3))))
+    if steps is None:  # size the timed region to about 2 s (a multiple of 20 steps)
+        t_ms, _, _ = g.timed(20, 3)
+        steps = int(min(20000, max(20, 2000.0 / max(t_ms / 20, 1e-3)))) // 20 * 20
     barrier(world)
     torch.cuda.synchronize(device)
     sampler = ClockSampler(device)

@@ -47,7 +47,7 @@ def test_plan_decode_invariants(lib):
         assert pl["path"] == 1
         assert pl["heads_per_cta"] == (64 if dk == 576 else 16)
         assert pl["head_blocks"] == -(-G // pl["heads_per_cta"])
-        ctas_per_sm = 2 if dk == 128 else 1
+        ctas_per_sm = 1 if dk == 576 else 2
         assert pl["kv_ranges"] == max(1, 148 * ctas_per_sm // pl["head_blocks"])
         assert pl["grid_ctas"] == pl["kv_ranges"] * pl["head_blocks"]
         assert pl["partials"] == pl["kv_ranges"] + B * Hkv
