@@ -122,8 +122,9 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
     pl->path = 0;
     pl->dv_parts = d_v / (d_v >= 512 ? 256 : 128);
     const int64_t n_qt = (Sq + 127) / 128;
-    pl->grid_ctas = n_qt * Hq * (int64_t)B * pl->dv_parts;
-    if (pl->grid_ctas > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
+    const int64_t items = n_qt * Hq * (int64_t)B * pl->dv_parts;  // persistent CTAs walk these
+    if (items > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
+    pl->grid_ctas = items < num_sms ? items : num_sms;
     pl->workspace_bytes = 0;
     return ATTN_OK;
   }
@@ -178,7 +179,7 @@ attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const
   using Tr = attn::PrefillTraits<DK, DVH>;
   auto kern = attn::prefill_kernel<DK, DVH, BF16>;
   set_smem(kern, Tr::SMEM_BYTES);
-  kern<<<(unsigned)pl.grid_ctas, 192, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
+  kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   return ATTN_OK;
 }
@@ -215,7 +216,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   if (reinterpret_cast<uintptr_t>(skv_per_seq) & 3u) return ATTN_EINVAL;
   if (!strides_ok(sq) || !strides_ok(sk) || !strides_ok(sv) || !strides_ok(so)) return ATTN_EINVAL;
   if (causal != 0 && causal != 1) return ATTN_EINVAL;
-  if (!std::isfinite(scale)) return ATTN_EINVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_EINVAL;
   attn_plan_t pl;
   attn_status_t rc = plan_impl(B, Hq, Hkv, Sq, max_skv, d_k, d_v, dtype, 0, &pl);
   if (rc != ATTN_OK) return rc;
@@ -294,6 +295,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.Sq = Sq;
   pp.n_qtiles = (Sq + 127) / 128;
   pp.dv_parts = pl.dv_parts;
+  pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;
   pp.scale_log2 = scale_log2;
   pp.causal = causal;
   pp.timeout_ns = kDefaultTimeoutNs;

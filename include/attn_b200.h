@@ -78,7 +78,7 @@ typedef struct {
                           CTA per range and head block                           */
   int64_t partials;    /* decode: partial-result slots (kv_ranges + B * Hkv)    */
   int dv_parts;        /* prefill: CTAs sharing one q tile, each owning d_v/dv_parts columns */
-  int64_t grid_ctas;   /* CTAs of the main kernel                               */
+  int64_t grid_ctas;   /* CTAs of the main kernel (persistent: at most one wave) */
   size_t workspace_bytes;
 } attn_plan_t;
 
@@ -106,7 +106,7 @@ size_t attn_workspace_bytes(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k
  *   skv_per_seq: device pointer, int32 [B], 0 <= skv[b] <= max_skv (not
  *                checked on the device).
  *   max_skv:     host value, the row extent of k and v (>= 1).
- *   scale:       multiplies q.k before the softmax (1/sqrt(d_k) for plain
+ *   scale:       > 0, multiplies q.k before the softmax (1/sqrt(d_k) for plain
  *                attention; 1/sqrt(192) for DeepSeek-V3 MLA, whose score
  *                scale follows the un-absorbed head width).
  *   causal:      0 or 1 (bottom-right alignment, see above).

@@ -112,9 +112,11 @@ def test_schedule_slots_unique_and_cover():
 def test_plan_prefill(lib):
     pl = binding.plan(2, 16, 1, 4096, 4096, 512, 512, num_sms=148)
     assert pl["path"] == 0 and pl["dv_parts"] == 2 and pl["workspace_bytes"] == 0
-    assert pl["grid_ctas"] == 32 * 16 * 2 * 2
+    assert pl["grid_ctas"] == 148  # persistent: one CTA per SM walks the 2048 work items
     pl = binding.plan(1, 64, 8, 8192, 8192, 128, 128, num_sms=148)
-    assert pl["dv_parts"] == 1 and pl["grid_ctas"] == 64 * 64
+    assert pl["dv_parts"] == 1 and pl["grid_ctas"] == 148
+    pl = binding.plan(1, 2, 1, 100, 100, 128, 128, num_sms=148)
+    assert pl["grid_ctas"] == 2  # fewer work items than SMs
 
 
 @pytest.mark.parametrize("args,code", [
@@ -154,6 +156,8 @@ def _call(lib, **over):
     (dict(sv=binding.Strides(-8, 0, 512)), binding.ATTN_EINVAL),
     (dict(causal=2), binding.ATTN_EINVAL),
     (dict(scale=float("nan")), binding.ATTN_EINVAL),
+    (dict(scale=-0.5), binding.ATTN_EINVAL),
+    (dict(scale=0.0), binding.ATTN_EINVAL),
     (dict(Hkv=3), binding.ATTN_EINVAL),
     (dict(dtype=7), binding.ATTN_EINVAL),
     (dict(d_k=64, d_v=64), binding.ATTN_EUNSUPPORTED),
