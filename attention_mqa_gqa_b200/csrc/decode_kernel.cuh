@@ -363,8 +363,9 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
         const uint64_t t0n = global_timer_ns();
         while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------ MMA issuer
+    } else if (warp == 1) {
+      // ------------------------------------------------ MMA issuer (whole warp,
+      // one elected lane issues; waits are polled by the converged warp)
       constexpr uint32_t idS = umma_idesc(128, NH, BF16, false, false);
       constexpr uint32_t idO = umma_idesc(128, NH, BF16, true, true);
       int slot = 0;
@@ -383,23 +384,29 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           if (!ok) return;
           tc_fence_after();
           const uint32_t abase = ring + slot * T::SLOT;
+          if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            // A = V^T: MN-major, 128-byte swizzle; the two 64-row halves of
-            // the 128-row block sit one slot apart (LBO); 8-key groups are
-            // 1024 bytes apart (SBO); 16 keys per K step = 2048 bytes.
-            const uint64_t ad = umma_sdesc(abase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
-            // B = P^T: MN-major, no swizzle; 8x8 core matrices, 8-head groups
-            // 128 bytes apart (SBO), 8-key groups NH*16 bytes apart (LBO).
-            const uint64_t bd = umma_sdesc(bbase + ks * 2 * NH * 16, NH * 16, 128, SMEM_NOSWIZZLE);
-            umma_ss(tmem + T::TMEM_O + i * NH, ad, bd, idO, (!first_of_piece || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 8; ++ks) {
+              // A = V^T: MN-major, 128-byte swizzle; the two 64-row halves of
+              // the 128-row block sit one slot apart (LBO); 8-key groups are
+              // 1024 bytes apart (SBO); 16 keys per K step = 2048 bytes.
+              const uint64_t ad = umma_sdesc(abase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
+              // B = P^T: MN-major, no swizzle; 8x8 core matrices, 8-head groups
+              // 128 bytes apart (SBO), 8-key groups NH*16 bytes apart (LBO).
+              const uint64_t bd =
+                  umma_sdesc(bbase + ks * 2 * NH * 16, NH * 16, 128, SMEM_NOSWIZZLE);
+              umma_ss(tmem + T::TMEM_O + i * NH, ad, bd, idO,
+                      (!first_of_piece || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(empty_bar(slot));
+            umma_commit(empty_bar(slot + 1));
           }
-          umma_commit(empty_bar(slot));
-          umma_commit(empty_bar(slot + 1));
+          __syncwarp();
           slot += 2;
           if (slot == T::RING) { slot = 0; ph ^= 1u; }
         }
-        umma_commit(o_done + 8 * pb);
+        if (elect_one()) umma_commit(o_done + 8 * pb);
+        __syncwarp();
       };
       PieceWalker w = walker();
       int b, kvh, t0, n, j = 0, k = 0;
@@ -422,27 +429,34 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
             tc_fence_after();
             const uint32_t abase = ring + slot * T::SLOT;
             const uint32_t bbase = qt + (k % T::NQ) * T::QT_BYTES + c * T::QT_CHUNK;
+            if (elect_one()) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
-              // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
-              const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
-              const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
-              umma_ss(tmem + T::TMEM_S + sb * NH, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks) {
+                // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
+                // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
+                const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
+                const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
+                umma_ss(tmem + T::TMEM_S + sb * NH, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+              }
+              umma_commit(empty_bar(slot));
             }
-            umma_commit(empty_bar(slot));
+            __syncwarp();
             if (++slot == T::RING) { slot = 0; ph ^= 1u; }
           }
           if (ok && T::KSLOTS > T::KCH) {
             ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 9);
             if (ok) {
-              mbar_arrive(empty_bar(slot));
+              if (elect_one()) mbar_arrive(empty_bar(slot));
+              __syncwarp();
               if (++slot == T::RING) { slot = 0; ph ^= 1u; }
             }
           }
           if (!ok) break;
-          umma_commit(s_full + 8 * sb);
-          if (i == n - 1) umma_commit(q_free + 8 * (k % T::NQ));  // this piece's Q^T is free
+          if (elect_one()) {
+            umma_commit(s_full + 8 * sb);
+            if (i == n - 1) umma_commit(q_free + 8 * (k % T::NQ));  // this piece's Q^T is free
+          }
+          __syncwarp();
           if (i > 0) pv(j - 1, prev_first);
           prev_first = (i == 0);
         }
@@ -451,7 +465,8 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
       if (ok && j > 0) pv(j - 1, prev_first);
       if (!ok) {
         // Gave up: let every MMA already issued finish before TMEM is freed.
-        umma_commit(drain);
+        if (elect_one()) umma_commit(drain);
+        __syncwarp();
         volatile int never = 0;
         mbar_wait(drain, 0, &never, 1000000ull, 10);
       }

@@ -229,8 +229,9 @@ __global__ void __launch_bounds__(64 + 256, 1)
       const uint64_t t0 = global_timer_ns();
       while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------- MMA issuer
+  } else if (warp == 1) {
+    // ---------------------------------------------------- MMA issuer (whole warp,
+    // one elected lane issues; waits are polled by the converged warp)
     constexpr uint32_t idS = umma_idesc(128, 128, BF16, false, false);  // Q, K both K-major
     constexpr uint32_t idO = umma_idesc(128, 128, BF16, false, true);   // P K-major, V MN-major
     int slot = 0;
@@ -252,22 +253,26 @@ __global__ void __launch_bounds__(64 + 256, 1)
         if (!ok) return;
         tc_fence_after();
         const uint32_t bbase = ring + slot * T::SLOT;
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          // A = P: K-major, 128-byte swizzle, keys 64*(ks/4) .. in chunk ks/4.
-          const uint64_t ad =
-              umma_sdesc(abase + (ks >> 2) * T::SLOT + (ks & 3) * 32, 16, 1024, SMEM_SW128);
-          // B = V: MN-major (d contiguous), 128-byte swizzle; the two 64-column
-          // halves are one slot apart (LBO), 8-key groups 1024 bytes (SBO).
-          const uint64_t bd = umma_sdesc(bbase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
-          umma_ss(tmem + T::TMEM_O + i * 128, ad, bd, idO, (!first || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < 8; ++ks) {
+            // A = P: K-major, 128-byte swizzle, keys 64*(ks/4) .. in chunk ks/4.
+            const uint64_t ad =
+                umma_sdesc(abase + (ks >> 2) * T::SLOT + (ks & 3) * 32, 16, 1024, SMEM_SW128);
+            // B = V: MN-major (d contiguous), 128-byte swizzle; the two 64-column
+            // halves are one slot apart (LBO), 8-key groups 1024 bytes (SBO).
+            const uint64_t bd = umma_sdesc(bbase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
+            umma_ss(tmem + T::TMEM_O + i * 128, ad, bd, idO, (!first || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(empty_bar(slot));
+          umma_commit(empty_bar(slot + 1));
         }
-        umma_commit(empty_bar(slot));
-        umma_commit(empty_bar(slot + 1));
+        __syncwarp();
         slot += 2;
         if (slot == T::RING) { slot = 0; ph ^= 1u; }
       }
-      umma_commit(o_done + 8 * pb);
+      if (elect_one()) umma_commit(o_done + 8 * pb);
+      __syncwarp();
     };
     int j = 0, kq = 0, prev_k = 0;
     bool prev_first = false;
@@ -291,18 +296,24 @@ __global__ void __launch_bounds__(64 + 256, 1)
           tc_fence_after();
           const uint32_t bbase = ring + slot * T::SLOT;
           const uint32_t abase = qs + qb * T::Q_BYTES + c * T::SLOT;
+          if (elect_one()) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
-            const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
-            umma_ss(tmem + T::TMEM_S + sb * 128, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
+              const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
+              umma_ss(tmem + T::TMEM_S + sb * 128, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(empty_bar(slot));
           }
-          umma_commit(empty_bar(slot));
+          __syncwarp();
           if (++slot == T::RING) { slot = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(s_full + 8 * sb);
-        if (i == it.ntiles - 1) umma_commit(q_free + 8 * qb);  // this item's Q is free
+        if (elect_one()) {
+          umma_commit(s_full + 8 * sb);
+          if (i == it.ntiles - 1) umma_commit(q_free + 8 * qb);  // this item's Q is free
+        }
+        __syncwarp();
         if (i > 0) pv(j - 1, prev_first, prev_k);
         prev_first = (i == 0);
         prev_k = kq;
@@ -311,7 +322,8 @@ __global__ void __launch_bounds__(64 + 256, 1)
     }
     if (ok && j > 0) pv(j - 1, prev_first, prev_k);
     if (!ok) {
-      umma_commit(drain);
+      if (elect_one()) umma_commit(drain);
+      __syncwarp();
       volatile int never = 0;
       mbar_wait(drain, 0, &never, 1000000ull, 29);
     }

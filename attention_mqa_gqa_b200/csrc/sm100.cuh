@@ -30,6 +30,18 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// One lane of the (converged) warp is elected; the warp stays converged.
+// Issuing tcgen05.mma / commit from an elected lane of a warp that runs the
+// whole control flow together keeps consecutive MMAs pipelined; a lone lane
+// that branches between MMAs (e.g. polling a barrier) issues them more slowly.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // 2^x on the SFU (PTX ex2.approx.ftz.f32: max relative error 2^-22 class).
 __device__ __forceinline__ float ex2(float x) {
   float y;
