@@ -162,7 +162,7 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
   if (phases & PHASE_PARTIAL) {
     auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
     set_smem(kern, Tr::SMEM_BYTES);
-    kern<<<(unsigned)pl.grid_ctas, 192, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
+    kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   if (phases & PHASE_COMBINE) {

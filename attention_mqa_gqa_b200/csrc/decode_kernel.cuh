@@ -28,10 +28,11 @@
 // [c_kv | k_pe] rows (d_k = 576) and V is the first 512 columns of the same
 // rows (d_v = 512), read through a second tensor map over the same memory.
 //
-// Warp roles (192 threads): warp 0 lane 0 streams K/V chunks through the
+// Warp roles (320 threads): warp 0 lane 0 streams K/V chunks through the
 // ring and lane 1 loads Q^T per piece (both TMA), warp 1 allocates TMEM and
-// issues UMMA, warps 2-5 run the softmax (thread = key row of the tile; for
-// O^T, thread = d_v row of each 128-row block) and the epilogues.
+// issues UMMA, warps 2-9 run the softmax and the epilogues: two threads per
+// key row of the tile (for O^T, per d_v row of each 128-row block), each
+// owning half of the group's heads.
 #pragma once
 
 #include "sm100.cuh"
@@ -64,8 +65,10 @@ struct DecodeTraits {
   static constexpr int VCH = DV / 64;              // 64-column V chunks per tile
   static constexpr int DVB = DV / 128;             // 128-row blocks of O^T
   static constexpr int CTAS = (DK == 576) ? 1 : 2; // resident CTAs per SM
-  static constexpr int RING = (DK == 576) ? 8 : (DK == 512 ? 4 : 6);
-  static constexpr int NPT = (DK == 576) ? 1 : 2;  // P^T buffers
+  static constexpr int RING = (DK == 576) ? 6 : (DK == 512 ? 4 : 6);
+  static constexpr int NPT = 2;                    // P^T buffers
+  static constexpr int SOFTMAX_THREADS = 256;      // two threads per key row
+  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr int NQ = (DK == 512) ? 2 : 1;   // Q^T buffers (next piece's Q^T prefetched)
   static constexpr int SLOT = 16384;               // one [128 x 64] 2-byte chunk
   static constexpr int QT_CHUNK = NH * 128;        // one [NH x 64] chunk of Q^T
@@ -205,7 +208,7 @@ __device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv,
 }
 
 template <int DK, int DV, int NH, bool BF16>
-__global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
+__global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTraits<DK, DV, NH>::CTAS)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
@@ -254,12 +257,12 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(s_free + 8 * i, 128);
-      mbar_init(red_full + 8 * i, 128);
+      mbar_init(s_free + 8 * i, T::SOFTMAX_THREADS);
+      mbar_init(red_full + 8 * i, T::SOFTMAX_THREADS);
       mbar_init(stat_ready + 8 * i, NH);
     }
     for (int i = 0; i < T::NPT; ++i) {
-      mbar_init(p_full + 8 * i, 128);
+      mbar_init(p_full + 8 * i, T::SOFTMAX_THREADS);
       mbar_init(o_done + 8 * i, 1);
     }
     for (int i = 0; i < T::NQ; ++i) {
@@ -472,12 +475,17 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
       }
     } else if (warp >= 2) {
       // ------------------------------------------------ softmax + epilogues
+      // Two threads per key row: warps w and w+4 share a TMEM lane quarter,
+      // each owning half (HH) of the group's heads for that key.
       // Cross-warp exchanges use mbarriers with bounded waits (red_full: all
-      // 128 partial values written; stat_ready: per-head statistics
-      // published), so a wait that gives up can never strand the other warps
-      // on a barrier.  These threads ignore the abort flag: all 128 wait on
+      // partial values written; stat_ready: per-head statistics published),
+      // so a wait that gives up can never strand the other warps on a
+      // barrier.  These threads ignore the abort flag: all of them wait on
       // the same barriers, so they either all see one complete or all time out.
-      const int st = threadIdx.x - 64;       // 0..127
+      constexpr int HH = NH / 2;
+      const int st = threadIdx.x - 64;       // 0..255
+      const int half = st >> 7;              // which half of the heads
+      const int h0l = half * HH;             // first head (of the NH) of this thread
       const int wq = warp & 3;               // TMEM lane quarter of this warp
       const int row = wq * 32 + lane;        // key row of S^T / d_v row of O^T blocks
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
@@ -486,7 +494,7 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
         return mbar_wait(bar, parity, &own_abort, p.timeout_ns, id);
       };
       if (st < NH) m_sm[st] = -INFINITY;
-      named_bar_sync(1, 128);
+      named_bar_sync(1, T::SOFTMAX_THREADS);
 
       PieceWalker w = walker();
       int b, kvh, t0, n, j = 0, r = 0;
@@ -494,9 +502,9 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
       while (ok && w.next(b, kvh, t0, n)) {
         const int skv_b = p.skv[b];
         const int64_t slot_id = (int64_t)rng + (int64_t)b * p.Hkv + kvh;  // workspace slot
-        float l[NH];
+        float l[HH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) l[h] = 0.f;
+        for (int h = 0; h < HH; ++h) l[h] = 0.f;
 
         for (int i = 0; i < n && ok; ++i, ++j, ++r) {
           const int sb = j & 1;
@@ -506,30 +514,27 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           if (!ok) break;
           tc_fence_after();
           const bool valid = (t0 + i) * T::TILE + row < skv_b;
-          // S^T row of this key (scaled to log2 units, masked), read from TMEM.
-          // It is read twice: once for the maxima and again for the weights,
-          // so that only one NH-wide array is live at a time.
-          auto load_s = [&](float (&x)[NH]) {
-#pragma unroll
-            for (int g = 0; g < NH / 16; ++g) {
-              float tmp[16];
-              tmem_ld16(tmem + lane_base + T::TMEM_S + sb * NH + g * 16, tmp);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) x[g * 16 + e] = valid ? tmp[e] * p.scale_log2 : -INFINITY;
-            }
+          // This thread's HH scores of its key (scaled to log2 units, masked),
+          // read from TMEM twice: for the maxima and again for the weights,
+          // so that only one HH-wide array is live at a time.
+          auto load_s = [&](float (&x)[HH]) {
+            tmem_ld<HH>(tmem + lane_base + T::TMEM_S + sb * NH + h0l, x);
             tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < HH; ++e) x[e] = valid ? x[e] * p.scale_log2 : -INFINITY;
           };
 
           // per-head maximum over the tile's 128 keys
           float* rbuf = red + rb * 4 * NH;
           {
-            float v[NH];
+            float v[HH];
             load_s(v);
-            transposed_warp_max<NH, NH, 16>(v, lane);
-            constexpr int HPL = NH >= 32 ? NH / 32 : 1;
-            if (NH >= 32 || (lane & (32 / NH - 1)) == 0) {
+            transposed_warp_max<HH, HH, 16>(v, lane);
+            constexpr int HPL = HH >= 32 ? HH / 32 : 1;
+            if (HH >= 32 || (lane & (32 / HH - 1)) == 0) {
 #pragma unroll
-              for (int e = 0; e < HPL; ++e) rbuf[wq * NH + transposed_head<NH>(lane, e)] = v[e];
+              for (int e = 0; e < HPL; ++e)
+                rbuf[wq * NH + h0l + transposed_head<HH>(lane, e)] = v[e];
             }
           }
           mbar_arrive(red_full + 8 * rb);
@@ -553,49 +558,56 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           ok = wait(stat_ready + 8 * rb, rpar, 13);
           if (!ok) break;
           const bool any = flags[rb] != 0;
+          // this thread's heads' running max and rescale factors (vector loads)
+          float mh[HH], ah[HH];
+#pragma unroll
+          for (int e = 0; e < HH; e += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(m_sm + h0l + e);
+            const float4 a4 = *reinterpret_cast<const float4*>(alpha_sm + h0l + e);
+            mh[e] = m4.x; mh[e + 1] = m4.y; mh[e + 2] = m4.z; mh[e + 3] = m4.w;
+            ah[e] = a4.x; ah[e + 1] = a4.y; ah[e + 2] = a4.z; ah[e + 3] = a4.w;
+          }
 
           const int pb = j % T::NPT;
           if (j >= T::NPT) {  // P^T buffer pb was last read by PV(j - NPT)
             ok = wait(o_done + 8 * pb, ((j - T::NPT) / T::NPT) & 1, 14);
             if (!ok) break;
           }
-          if (any && i > 0) {  // rescale O^T once PV(j-1) has landed
+          if (any && i > 0) {  // rescale this thread's O^T columns once PV(j-1) has landed
             ok = wait(o_done + 8 * ((j - 1) % T::NPT), ((j - 1) / T::NPT) & 1, 15);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll 1
             for (int d = 0; d < T::DVB; ++d) {
+              float o[HH];
+              const uint32_t ta = tmem + lane_base + T::TMEM_O + d * NH + h0l;
+              tmem_ld<HH>(ta, o);
+              tmem_wait_ld();
 #pragma unroll
-              for (int g = 0; g < NH / 16; ++g) {
-                float o[16];
-                const uint32_t ta = tmem + lane_base + T::TMEM_O + d * NH + g * 16;
-                tmem_ld16(ta, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 16; ++c) o[c] *= alpha_sm[g * 16 + c];
-                tmem_st16(ta, o);
-              }
+              for (int c = 0; c < HH; ++c) o[c] *= ah[c];
+              tmem_st<HH>(ta, o);
             }
             tmem_wait_st();
           }
 #pragma unroll
-          for (int h = 0; h < NH; ++h) l[h] *= alpha_sm[h];
+          for (int h = 0; h < HH; ++h) l[h] *= ah[h];
 
-          float s[NH];
-          load_s(s);
+          float sv[HH];
+          load_s(sv);
           tc_fence_before();
           mbar_arrive(s_free + 8 * sb);
 
-          // P^T row for this key: NH values, written as MN-major core matrices.
-          const uint32_t prow = pt + pb * T::PT_BYTES + (row >> 3) * (NH * 16) + (row & 7) * 16;
+          // P^T row for this key, this thread's HH heads, as MN-major core matrices.
+          const uint32_t prow = pt + pb * T::PT_BYTES + (row >> 3) * (NH * 16) + (row & 7) * 16 +
+                                (h0l >> 3) * 128;
 #pragma unroll
-          for (int g = 0; g < NH / 8; ++g) {
+          for (int g = 0; g < HH / 8; ++g) {
             uint32_t u[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int h = g * 8 + 2 * e;
-              const float p0 = s[h] == -INFINITY ? 0.f : ex2(s[h] - m_sm[h]);
-              const float p1 = s[h + 1] == -INFINITY ? 0.f : ex2(s[h + 1] - m_sm[h + 1]);
+              const float p0 = sv[h] == -INFINITY ? 0.f : ex2(sv[h] - mh[h]);
+              const float p1 = sv[h + 1] == -INFINITY ? 0.f : ex2(sv[h + 1] - mh[h + 1]);
               u[e] = pack2(p0, p1, BF16);
               l[h] += p0;
               l[h + 1] += p1;
@@ -618,11 +630,11 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           const uint32_t rpar = (r >> 1) & 1;
           float* rbuf = red + rb * 4 * NH;
 #pragma unroll
-          for (int h = 0; h < NH; ++h) {
+          for (int h = 0; h < HH; ++h) {
             float v = l[h];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) rbuf[wq * NH + h] = v;
+            if (lane == 0) rbuf[wq * NH + h0l + h] = v;
           }
           mbar_arrive(red_full + 8 * rb);
           ok = wait(red_full + 8 * rb, rpar, 17);
@@ -642,19 +654,16 @@ __global__ void __launch_bounds__(192, DecodeTraits<DK, DV, NH>::CTAS)
           ++r;
 #pragma unroll 1
           for (int d = 0; d < T::DVB; ++d) {
+            float o[HH];
+            tmem_ld<HH>(tmem + lane_base + T::TMEM_O + d * NH + h0l, o);
+            tmem_wait_ld();
+            const int dd = d * 128 + row;
 #pragma unroll
-            for (int g = 0; g < NH / 16; ++g) {
-              float o[16];
-              tmem_ld16(tmem + lane_base + T::TMEM_O + d * NH + g * 16, o);
-              tmem_wait_ld();
-              const int dd = d * 128 + row;
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int h = g * 16 + c;
-                if (h < nvalid) {
-                  const float L = l_sm[h];
-                  p.ws_o[(slot_id * p.G + hb * NH + h) * DV + dd] = L > 0.f ? o[c] / L : 0.f;
-                }
+            for (int c = 0; c < HH; ++c) {
+              const int h = h0l + c;
+              if (h < nvalid) {
+                const float L = l_sm[h];
+                p.ws_o[(slot_id * p.G + hb * NH + h) * DV + dd] = L > 0.f ? o[c] / L : 0.f;
               }
             }
           }

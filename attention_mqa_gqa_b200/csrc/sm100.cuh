@@ -213,6 +213,62 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) 
       : "memory");
 }
 
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
+  uint32_t u[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]),
+                 "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(__float_as_uint(r[0])), "r"(__float_as_uint(r[1])), "r"(__float_as_uint(r[2])),
+               "r"(__float_as_uint(r[3])), "r"(__float_as_uint(r[4])), "r"(__float_as_uint(r[5])),
+               "r"(__float_as_uint(r[6])), "r"(__float_as_uint(r[7]))
+               : "memory");
+}
+
+// Load/store `N` (a multiple of 8) consecutive columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&r)[N]) {
+  static_assert(N % 8 == 0, "columns");
+#pragma unroll
+  for (int g = 0; g < N / 16; ++g) {
+    float t[16];
+    tmem_ld16(taddr + g * 16, t);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[g * 16 + i] = t[i];
+  }
+  if constexpr (N % 16 != 0) {
+    float t[8];
+    tmem_ld8(taddr + (N / 16) * 16, t);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[(N / 16) * 16 + i] = t[i];
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&r)[N]) {
+  static_assert(N % 8 == 0, "columns");
+#pragma unroll
+  for (int g = 0; g < N / 16; ++g) {
+    float t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t[i] = r[g * 16 + i];
+    tmem_st16(taddr + g * 16, t);
+  }
+  if constexpr (N % 16 != 0) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = r[(N / 16) * 16 + i];
+    tmem_st8(taddr + (N / 16) * 16, t);
+  }
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
