@@ -42,7 +42,7 @@ class AttnError(RuntimeError):
 # Every symbol include/attn_b200.h declares (checked by the CPU test suite).
 EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
            "attn_decode_combine", "attn_fwd_noalloc", "attn_last_device_error", "attn_status_str",
-           "attn_version")
+           "attn_version", "attn_set_wait_timeout_ns")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in the header
 
 _lib = None
@@ -71,6 +71,8 @@ def load(path: str | None = None):
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
                                      ctypes.c_float, i32, i32, Strides, Strides, Strides,
                                      Strides, vp]
+    lib.attn_set_wait_timeout_ns.restype = ctypes.c_uint64
+    lib.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.attn_last_device_error.restype = i32
     lib.attn_last_device_error.argtypes = [vp]
     lib.attn_status_str.restype = ctypes.c_char_p
@@ -181,6 +183,12 @@ def attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: tor
 def last_device_error(stream: torch.cuda.Stream | None = None) -> int:
     st = stream if stream is not None else torch.cuda.current_stream()
     return int(load().attn_last_device_error(st.cuda_stream))
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    """Bound every device-side wait of later launches (0 = default 2 s);
+    returns the previous bound.  Diagnostic only (see the header)."""
+    return int(load().attn_set_wait_timeout_ns(int(ns)))
 
 
 def attention(q, k, v, skv, max_skv, scale, causal=True, with_lse=True, workspace=None,

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/attn_b200.h"
@@ -19,6 +20,7 @@
 namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+std::atomic<uint64_t> g_wait_timeout_ns{kDefaultTimeoutNs};  // read at each launch
 
 // ------------------------------------------------------------------ driver
 
@@ -254,7 +256,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     dp.ranges = pl.kv_ranges;
     dp.head_blocks = pl.head_blocks;
     dp.scale_log2 = scale_log2;
-    dp.timeout_ns = kDefaultTimeoutNs;
+    dp.timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);
     attn::CombineParams cp{};
     cp.ws_o = dp.ws_o;
     cp.ws_lse = dp.ws_lse;
@@ -298,7 +300,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;
   pp.scale_log2 = scale_log2;
   pp.causal = causal;
-  pp.timeout_ns = kDefaultTimeoutNs;
+  pp.timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);
   if (d_k == 128)
     return bf16 ? launch_prefill<128, 128, true>(mq, mk, mv, pp, pl, st)
                 : launch_prefill<128, 128, false>(mq, mk, mv, pp, pl, st);
@@ -365,6 +367,10 @@ const char* attn_status_str(attn_status_t s) {
 }
 
 const char* attn_version(void) { return "0.1.0"; }
+
+uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
+  return g_wait_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);
+}
 
 }  // extern "C"
 

@@ -340,10 +340,6 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
         }
       }
       if (pv_tok >= 0) load_v();
-      if (!ok) {  // give issued copies time to land before the CTA leaves
-        const uint64_t t0n = global_timer_ns();
-        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
-      }
     } else if (warp == 0 && lane == 1) {
       // ------------------------------------------------ producer: Q^T per piece
       tma_prefetch_desc(&tmQ);
@@ -362,10 +358,6 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
                       kvh * p.G + hb * NH, b, pol);
         ++k;
       }
-      if (!ok) {
-        const uint64_t t0n = global_timer_ns();
-        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
-      }
     } else if (warp == 1) {
       // ------------------------------------------------ MMA issuer (whole warp,
       // one elected lane issues; waits are polled by the converged warp)
@@ -377,30 +369,29 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       auto pv = [&](int t, bool first_of_piece) {
         if (!ok) return;
         const int pb = t % T::NPT;
-        ok = mbar_wait(p_full + 8 * pb, (t / T::NPT) & 1, abort_flag, p.timeout_ns, 4);
+        ok = mbar_wait_warp(p_full + 8 * pb, (t / T::NPT) & 1, abort_flag, p.timeout_ns, 4);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t bbase = pt + pb * T::PT_BYTES;
+        // B = P^T: MN-major, no swizzle; 8x8 core matrices, 8-head groups 128
+        // bytes apart (SBO), 8-key groups NH*16 bytes apart (LBO); 16 keys per
+        // K step = 2*NH*16 bytes.
+        const uint64_t bd0 = umma_sdesc(pt + pb * T::PT_BYTES, NH * 16, 128, SMEM_NOSWIZZLE);
         for (int i = 0; i < T::DVB; ++i) {
-          ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 5) &&
-               mbar_wait(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 5);
+          ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 5) &&
+               mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 5);
           if (!ok) return;
           tc_fence_after();
-          const uint32_t abase = ring + slot * T::SLOT;
           if (elect_one()) {
+            // A = V^T: MN-major, 128-byte swizzle; the two 64-row halves of
+            // the 128-row block sit one slot apart (LBO); 8-key groups are
+            // 1024 bytes apart (SBO); 16 keys per K step = 2048 bytes.
+            const uint64_t ad0 = umma_sdesc(ring + slot * T::SLOT, T::SLOT, 1024, SMEM_SW128);
+            const uint32_t d = tmem + T::TMEM_O + i * NH;
+            umma_ss(d, ad0, bd0, idO, first_of_piece ? 0u : 1u);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              // A = V^T: MN-major, 128-byte swizzle; the two 64-row halves of
-              // the 128-row block sit one slot apart (LBO); 8-key groups are
-              // 1024 bytes apart (SBO); 16 keys per K step = 2048 bytes.
-              const uint64_t ad = umma_sdesc(abase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
-              // B = P^T: MN-major, no swizzle; 8x8 core matrices, 8-head groups
-              // 128 bytes apart (SBO), 8-key groups NH*16 bytes apart (LBO).
-              const uint64_t bd =
-                  umma_sdesc(bbase + ks * 2 * NH * 16, NH * 16, 128, SMEM_NOSWIZZLE);
-              umma_ss(tmem + T::TMEM_O + i * NH, ad, bd, idO,
-                      (!first_of_piece || ks > 0) ? 1u : 0u);
-            }
+            for (int ks = 1; ks < 8; ++ks)
+              umma_ss(d, ad0 + (uint64_t)(ks * (2048 >> 4)), bd0 + (uint64_t)(ks * (2 * NH * 16 >> 4)),
+                      idO, 1u);
             umma_commit(empty_bar(slot));
             umma_commit(empty_bar(slot + 1));
           }
@@ -419,40 +410,43 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
           const int sb = j & 1;
           if (i == 0 && j > 0) pv(j - 1, prev_first);  // finish the previous piece first
           if (i == 0) {
-            ok = ok && mbar_wait(q_full + 8 * (k % T::NQ), (k / T::NQ) & 1, abort_flag, p.timeout_ns, 6);
+            ok = ok && mbar_wait_warp(q_full + 8 * (k % T::NQ), (k / T::NQ) & 1, abort_flag, p.timeout_ns, 6);
             if (!ok) break;
             tc_fence_after();
           }
-          if (j >= 2) ok = mbar_wait(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 7);
+          if (j >= 2) ok = mbar_wait_warp(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 7);
           if (!ok) break;
           tc_fence_after();
-          for (int c = 0; c < T::KCH && ok; ++c) {
-            ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 8);
+          // K chunks are consumed in pairs (two ring slots, eight MMAs per
+          // wait); with an odd chunk count the last pair's second slot is the
+          // producer's empty placeholder.
+          const uint32_t qbase = qt + (k % T::NQ) * T::QT_BYTES;
+          for (int c = 0; c < T::KCH && ok; c += 2) {
+            ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 8) &&
+                 mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 8);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t abase = ring + slot * T::SLOT;
-            const uint32_t bbase = qt + (k % T::NQ) * T::QT_BYTES + c * T::QT_CHUNK;
             if (elect_one()) {
+              // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
+              // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
+              const uint64_t ad0 = umma_sdesc(ring + slot * T::SLOT, 16, 1024, SMEM_SW128);
+              const uint64_t bd0 = umma_sdesc(qbase + c * T::QT_CHUNK, 16, 1024, SMEM_SW128);
+              const uint32_t d = tmem + T::TMEM_S + sb * NH;
+              umma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
-                // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
-                const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
-                const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
-                umma_ss(tmem + T::TMEM_S + sb * NH, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 1; ks < 4; ++ks) umma_ss(d, ad0 + 2 * ks, bd0 + 2 * ks, idS, 1u);
+              if (c + 1 < T::KCH) {
+                const uint64_t ad1 = ad0 + (T::SLOT >> 4);
+                const uint64_t bd1 = bd0 + (T::QT_CHUNK >> 4);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) umma_ss(d, ad1 + 2 * ks, bd1 + 2 * ks, idS, 1u);
               }
               umma_commit(empty_bar(slot));
+              umma_commit(empty_bar(slot + 1));
             }
             __syncwarp();
-            if (++slot == T::RING) { slot = 0; ph ^= 1u; }
-          }
-          if (ok && T::KSLOTS > T::KCH) {
-            ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 9);
-            if (ok) {
-              if (elect_one()) mbar_arrive(empty_bar(slot));
-              __syncwarp();
-              if (++slot == T::RING) { slot = 0; ph ^= 1u; }
-            }
+            slot += 2;
+            if (slot == T::RING) { slot = 0; ph ^= 1u; }
           }
           if (!ok) break;
           if (elect_one()) {
@@ -466,13 +460,6 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
         ++k;
       }
       if (ok && j > 0) pv(j - 1, prev_first);
-      if (!ok) {
-        // Gave up: let every MMA already issued finish before TMEM is freed.
-        if (elect_one()) umma_commit(drain);
-        __syncwarp();
-        volatile int never = 0;
-        mbar_wait(drain, 0, &never, 1000000ull, 10);
-      }
     } else if (warp >= 2) {
       // ------------------------------------------------ softmax + epilogues
       // Two threads per key row: warps w and w+4 share a TMEM lane quarter,
@@ -491,7 +478,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
       volatile int own_abort = 0;
       auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
-        return mbar_wait(bar, parity, &own_abort, p.timeout_ns, id);
+        return mbar_wait_warp(bar, parity, &own_abort, p.timeout_ns, id);
       };
       if (st < NH) m_sm[st] = -INFINITY;
       named_bar_sync(1, T::SOFTMAX_THREADS);
@@ -673,6 +660,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       if (!ok) *abort_flag = 1;
     }
   }
+  abort_tail(abort_flag, warp, drain);
 
   tc_fence_before();
   __syncthreads();

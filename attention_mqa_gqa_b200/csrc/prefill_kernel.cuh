@@ -202,10 +202,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
       }
     }
     if (have_prev) load_v();
-    if (!ok) {  // give issued copies time to land before the CTA leaves
-      const uint64_t t0 = global_timer_ns();
-      while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
-    }
   } else if (warp == 0 && lane == 1) {
     // ---------------------------------------------------- producer: Q per item
     tma_prefetch_desc(&tmQ);
@@ -225,10 +221,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
                     it.h, it.b, pol_q);
       ++kq;
     }
-    if (!ok) {
-      const uint64_t t0 = global_timer_ns();
-      while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
-    }
   } else if (warp == 1) {
     // ---------------------------------------------------- MMA issuer (whole warp,
     // one elected lane issues; waits are polled by the converged warp)
@@ -242,14 +234,14 @@ __global__ void __launch_bounds__(64 + 256, 1)
     auto pv = [&](int t, bool first, int k) {
       if (!ok) return;
       const int pb = t % T::NPBUF;
-      ok = mbar_wait(p_full + 8 * pb, (t / T::NPBUF) & 1, abort_flag, p.timeout_ns, 23);
-      if (ok && first && k > 0) ok = mbar_wait(o_free, (k - 1) & 1, abort_flag, p.timeout_ns, 24);
+      ok = mbar_wait_warp(p_full + 8 * pb, (t / T::NPBUF) & 1, abort_flag, p.timeout_ns, 23);
+      if (ok && first && k > 0) ok = mbar_wait_warp(o_free, (k - 1) & 1, abort_flag, p.timeout_ns, 24);
       if (!ok) return;
       tc_fence_after();
       const uint32_t abase = ps + pb * T::P_BYTES;
       for (int i = 0; i < T::VCH / 2; ++i) {
-        ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 25) &&
-             mbar_wait(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 25);
+        ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 25) &&
+             mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 25);
         if (!ok) return;
         tc_fence_after();
         const uint32_t bbase = ring + slot * T::SLOT;
@@ -284,14 +276,14 @@ __global__ void __launch_bounds__(64 + 256, 1)
         const int sb = j & 1;
         if (i == 0 && j > 0) pv(j - 1, prev_first, prev_k);  // finish the previous item
         if (i == 0) {
-          ok = ok && mbar_wait(q_full + 8 * qb, (kq / T::NQ) & 1, abort_flag, p.timeout_ns, 26);
+          ok = ok && mbar_wait_warp(q_full + 8 * qb, (kq / T::NQ) & 1, abort_flag, p.timeout_ns, 26);
           if (!ok) break;
         }
-        if (j >= 2) ok = mbar_wait(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 27);
+        if (j >= 2) ok = mbar_wait_warp(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 27);
         if (!ok) break;
         tc_fence_after();
         for (int c = 0; c < T::KCH && ok; ++c) {
-          ok = mbar_wait(full_bar(slot), ph, abort_flag, p.timeout_ns, 28);
+          ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 28);
           if (!ok) break;
           tc_fence_after();
           const uint32_t bbase = ring + slot * T::SLOT;
@@ -321,12 +313,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
       ++kq;
     }
     if (ok && j > 0) pv(j - 1, prev_first, prev_k);
-    if (!ok) {
-      if (elect_one()) umma_commit(drain);
-      __syncwarp();
-      volatile int never = 0;
-      mbar_wait(drain, 0, &never, 1000000ull, 29);
-    }
   } else if (warp >= 2) {
     // ---------------------------------------------------- softmax + epilogue
     const int wq = warp & 3;
@@ -334,15 +320,20 @@ __global__ void __launch_bounds__(64 + 256, 1)
     const int row = wq * 32 + lane;          // q row within the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     constexpr int HC = DVH / 2;              // output columns per thread
-    // the two threads of a row meet on named barrier 1 + wq (warps w, w + 4)
+    // The two threads of a row meet on named barrier 1 + wq (warps w, w + 4).
+    // A pair barrier waits without bound, so both threads must always reach
+    // the same ones: a failed wait only clears `ok` (skipping the work that
+    // depends on it), and the pair leaves its loops together right after the
+    // next pair barrier that ANDs `ok` over both (pair_and).
     auto pair_sync = [&]() { named_bar_sync(1 + wq, 64); };
+    auto pair_and = [&](bool v) { return named_bar_and(1 + wq, 64, v); };
     volatile int own_abort = 0;
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
-      return mbar_wait(bar, parity, &own_abort, p.timeout_ns, id);
+      return mbar_wait_warp(bar, parity, &own_abort, p.timeout_ns, id);
     };
     bool ok = true;
     int j = 0;
-    for (int L = blockIdx.x; L < p.n_items && ok; L += gridDim.x) {
+    for (int L = blockIdx.x; L < p.n_items; L += gridDim.x) {
       const PrefillItem it = prefill_item(p, L);
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
@@ -350,34 +341,33 @@ __global__ void __launch_bounds__(64 + 256, 1)
       float m_used = -INFINITY;  // log2-domain running max (lazily raised), same in both halves
       float l = 0.f;             // this half's share of the row sum
 
-      for (int i = 0; i < it.ntiles && ok; ++i, ++j) {
+      for (int i = 0; i < it.ntiles; ++i, ++j) {
         const int sb = j & 1;
-        ok = wait(s_full + 8 * sb, (j >> 1) & 1, 30);
-        if (!ok) break;
-        tc_fence_after();
+        if (ok) ok = wait(s_full + 8 * sb, (j >> 1) & 1, 30);
         float s[64];
+        float mx = -INFINITY;
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float tmp[16];
-          tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + half * 64 + g * 16, tmp);
+          for (int g = 0; g < 4; ++g) {
+            float tmp[16];
+            tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + half * 64 + g * 16, tmp);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_free + 8 * sb);
+            for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
+          }
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(s_free + 8 * sb);
 
-        const int kb = i * T::KT + half * 64;
-        // Keys at or past `lim` are invisible to this row; only tiles that
-        // straddle `lim` need the mask.  The maximum is taken on the raw
-        // scores (scale > 0) in 8 independent chains, then scaled once.
-        if (kb + 64 > lim) {
+          const int kb = i * T::KT + half * 64;
+          // Keys at or past `lim` are invisible to this row; only tiles that
+          // straddle `lim` need the mask.  The maximum is taken on the raw
+          // scores (scale > 0) in 8 independent chains, then scaled once.
+          if (kb + 64 > lim) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (kb + c >= lim) s[c] = -INFINITY;
-        }
-        float mx;
-        {
+            for (int c = 0; c < 64; ++c)
+              if (kb + c >= lim) s[c] = -INFINITY;
+          }
           float mc[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) mc[e] = s[e];
@@ -390,7 +380,8 @@ __global__ void __launch_bounds__(64 + 256, 1)
         // buffer alternates with the tile so one barrier per tile suffices)
         float* xb = xch + (j & 1) * 128;
         if (half == 1) xb[row] = mx;
-        pair_sync();
+        ok = pair_and(ok);
+        if (!ok) break;
         if (half == 0) mx = fmaxf(mx, xb[row]);
         if (half == 0) xb[row] = mx;
         pair_sync();
@@ -403,14 +394,14 @@ __global__ void __launch_bounds__(64 + 256, 1)
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
         const bool warp_need = __any_sync(0xffffffffu, need);
         const int pb = j % T::NPBUF;
-        if (j >= T::NPBUF) {  // P buffer pb was last read by PV(j - NPBUF)
-          ok = wait(o_done + 8 * pb, ((j - T::NPBUF) / T::NPBUF) & 1, 31);
-          if (!ok) break;
-        }
+        // P buffer pb was last read by PV(j - NPBUF); a failed wait ends the
+        // tile here and the pair leaves at the next pair_and
+        if (j >= T::NPBUF) ok = wait(o_done + 8 * pb, ((j - T::NPBUF) / T::NPBUF) & 1, 31);
+        if (!ok) continue;
         if (warp_need && i > 0) {  // rescale this thread's O columns once PV(j-1) landed
           const int t = j - 1;
           ok = wait(o_done + 8 * (t % T::NPBUF), (t / T::NPBUF) & 1, 32);
-          if (!ok) break;
+          if (!ok) continue;
           tc_fence_after();
 #pragma unroll 1
           for (int g = 0; g < HC / 16; ++g) {
@@ -455,14 +446,14 @@ __global__ void __launch_bounds__(64 + 256, 1)
         tc_fence_before();
         mbar_arrive(p_full + 8 * pb);
       }
-      if (!ok) break;
 
       // ------------------------------------------------------ epilogue
       // row sum = both halves (the exchange buffer of this round is free:
       // its last readers passed the second pair barrier of the last tile)
       float* xb = xch + (j & 1) * 128;
       if (half == 1) xb[row] = l;
-      pair_sync();
+      ok = pair_and(ok);
+      if (!ok) break;
       const float lrow = half == 0 ? l + xb[row] : 0.f;
       if (half == 0) xb[row] = lrow;
       pair_sync();
@@ -470,7 +461,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
       if (it.ntiles > 0) {
         const int t = j - 1;
         ok = wait(o_done + 8 * (t % T::NPBUF), (t / T::NPBUF) & 1, 33);
-        if (!ok) break;
+        if (!ok) continue;  // no pair barrier before the next item's first pair_and
         tc_fence_after();
       }
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
@@ -506,6 +497,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
     }
     if (!ok) *abort_flag = 1;
   }
+  abort_tail(abort_flag, warp, drain);
 
   tc_fence_before();
   __syncthreads();

@@ -30,6 +30,21 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier that also ANDs a predicate over its `nthreads` threads:
+// every participant returns true only if all of them passed true.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, p;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // One lane of the (converged) warp is elected; the warp stays converged.
 // Issuing tcgen05.mma / commit from an elected lane of a warp that runs the
 // whole control flow together keeps consecutive MMAs pipelined; a lone lane
@@ -91,18 +106,41 @@ __device__ unsigned int g_attn_error;
 // false.  Never traps and never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns, uint32_t id) {
+  // try_wait itself suspends the thread for a while before it reports an
+  // incomplete phase, so the clock and the abort flag are checked after
+  // every unsuccessful poll.
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicCAS(&g_attn_error, 0u, 1u | ((id & 0xffu) << 8));
+      atomicOr(&g_attn_error, 1u);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// mbar_wait for a whole converged warp: every lane returns the same value
+// (the votes keep the warp converged for the shuffles, elect.sync and
+// tcgen05 collectives that follow a wait, also when the wait gives up).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint64_t timeout_ns, uint32_t id) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    const bool aborted = __any_sync(0xffffffffu, *abort != 0);
+    const bool late = __any_sync(0xffffffffu, global_timer_ns() - t0 > timeout_ns);
+    if (aborted || late) {
+      if (late && (threadIdx.x & 31u) == 0) {
         atomicCAS(&g_attn_error, 0u, 1u | ((id & 0xffu) << 8));
         atomicOr(&g_attn_error, 1u);
-        *abort = 1;
-        return false;
       }
+      *abort = 1;
+      return false;
     }
   }
 }
@@ -319,6 +357,27 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
       : "memory");
+}
+
+// Common exit of the warp-specialised kernels, called by every thread once
+// all roles have left their loops.  If any wait gave up (abort flag set),
+// copies already issued by the producers and MMAs already issued by warp 1
+// must complete before the CTA releases its shared memory and TMEM: warp 1
+// commits the `drain` barrier and waits for it (bounded), thread 0 gives
+// in-flight TMA copies 2 ms to land.
+__device__ __forceinline__ void abort_tail(volatile int* abort_flag, int warp, uint32_t drain) {
+  __syncthreads();
+  if (*abort_flag == 0) return;
+  if (warp == 1) {
+    if (elect_one()) umma_commit(drain);
+    __syncwarp();
+    volatile int never = 0;
+    mbar_wait_warp(drain, 0, &never, 1000000ull, 30);
+  }
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+  }
 }
 
 // ---------------------------------------------------------------- layouts

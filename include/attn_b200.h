@@ -185,6 +185,15 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void
  */
 attn_status_t attn_last_device_error(void* cuda_stream);
 
+/* Bound on every device-side wait of launches made after this call, in
+ * nanoseconds of %globaltimer (process-wide; 0 restores the default of 2 s).
+ * Returns the previous bound.  A diagnostic: a bound far below a kernel's
+ * normal waiting times makes its waits give up, so the error path (abort,
+ * drain, ATTN_ETIMEOUT from attn_last_device_error) can be exercised without
+ * any fault.  The pages have no counterpart.  Not synchronised with launches
+ * running on other host threads. */
+uint64_t attn_set_wait_timeout_ns(uint64_t ns);
+
 /* Static, human-readable name of a status code. */
 const char* attn_status_str(attn_status_t status);
 
