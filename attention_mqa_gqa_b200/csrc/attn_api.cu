@@ -43,22 +43,27 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B, H, S, D] tensor (innermost D), box = 64 columns x 128
-// rows, 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t S,
-              uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb) {
+// 5-D map over a [B, H, S, D] tensor that splits each row into D/64 chunks
+// of 64 columns: dims (innermost first) = {64, S, D/64, H, B} with the chunk
+// dimension's stride 128 bytes, box = 64 columns x 128 rows x `kch` chunks,
+// 128-byte swizzle.  One copy thus lands `kch` consecutive [128 x 64]
+// chunk tiles, each in the layout a per-chunk 2-D box would give, so a
+// single TMA instruction moves kch * 16 KB (a copy stream of 16 KB boxes is
+// limited per CTA well below HBM bandwidth).  D must be a multiple of 64;
+// chunks past D/64 are out of range and zero-filled.
+bool make_chunk_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t S,
+                    uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb, uint32_t kch) {
   EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  // strides of extent-1 dimensions are irrelevant; give them valid values
+  if (!enc || D % 64 != 0) return false;
   if (S == 1) ss = (int64_t)D;
   if (H == 1) sh = ss * (int64_t)S;
   if (B == 1) sb = sh * (int64_t)H;
-  cuuint64_t dims[4] = {D, S, H, B};
-  cuuint64_t strides[3] = {(cuuint64_t)ss * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
+  cuuint64_t dims[5] = {64, S, D / 64, H, B};
+  cuuint64_t strides[4] = {(cuuint64_t)ss * 2, 128, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  cuuint32_t box[5] = {64, 128, kch, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   4, const_cast<void*>(base), dims, strides, box, estr,
+                   5, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -235,11 +240,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   const int G = Hq / Hkv;
 
   CUtensorMap mk, mv;
-  if (!make_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b)) return ATTN_ECUDA;
-  if (!make_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b)) return ATTN_ECUDA;
-
   if (pl.path == 1) {
     if ((Hq > 1 && sq.h == 0) || (B > 1 && sq.b == 0)) return ATTN_EINVAL;
+    if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;
+    if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
     CUtensorMap mq;
     if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, (uint32_t)pl.heads_per_cta))
       return ATTN_ECUDA;
@@ -281,8 +285,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
                 : launch_decode<576, 512, 64, false>(mq, mk, mv, dp, cp, pl, st, phases);
   }
 
+  if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;
+  if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
   CUtensorMap mq;
-  if (!make_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b)) return ATTN_ECUDA;
+  if (!make_chunk_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b, 2)) return ATTN_ECUDA;
   attn::PrefillParams pp{};
   pp.out = out;
   pp.o_sb = so.b;

@@ -61,8 +61,14 @@ template <int DK, int DV, int NH>
 struct DecodeTraits {
   static constexpr int TILE = 128;                 // keys per tile (MMA M)
   static constexpr int KCH = DK / 64;              // 64-column K chunks per tile
-  static constexpr int KSLOTS = (KCH + 1) & ~1;    // ring slots per tile's K (even)
   static constexpr int VCH = DV / 64;              // 64-column V chunks per tile
+  // One TMA copy moves GCH consecutive chunks of a tile into one ring group
+  // (a single copy of 16 KB per chunk caps a CTA's stream well below HBM
+  // bandwidth).  With an odd chunk count the last K group's second chunk
+  // lies past the row's end and is zero-filled by the copy.
+  static constexpr int GCH = 2;
+  static constexpr int KG = (KCH + GCH - 1) / GCH;  // ring groups per K tile
+  static constexpr int VG = VCH / GCH;              // ring groups per V tile (one per O^T block)
   static constexpr int DVB = DV / 128;             // 128-row blocks of O^T
   static constexpr int CTAS = (DK == 576) ? 1 : 2; // resident CTAs per SM
   static constexpr int RING = (DK == 576) ? 6 : (DK == 512 ? 4 : 6);
@@ -71,6 +77,8 @@ struct DecodeTraits {
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr int NQ = (DK == 512) ? 2 : 1;   // Q^T buffers (next piece's Q^T prefetched)
   static constexpr int SLOT = 16384;               // one [128 x 64] 2-byte chunk
+  static constexpr int GBYTES = GCH * SLOT;         // one ring group
+  static constexpr int RING_G = RING / GCH;         // ring groups
   static constexpr int QT_CHUNK = NH * 128;        // one [NH x 64] chunk of Q^T
   static constexpr int PT_BYTES = NH * TILE * 2;   // one P^T buffer
   static constexpr int OFF_RING = 0;
@@ -85,16 +93,16 @@ struct DecodeTraits {
   static constexpr int OFF_SCHED = OFF_SCAN + 64;               // int [4] range start
   static constexpr int OFF_FLAGS = OFF_SCHED + 16;              // int [4]: any[2], abort, tmem
   static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
-  // full[RING], empty[RING], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full[NQ],
+  // full[RING_G], empty[RING_G], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full[NQ],
   // q_free[NQ], red_full[2], stat_ready[2], drain
-  static constexpr int NBAR = 2 * RING + 9 + 2 * NPT + 2 * NQ;
+  static constexpr int NBAR = 2 * RING_G + 9 + 2 * NPT + 2 * NQ;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;  // + alignment slack
   static constexpr int TMEM_S = 0;                  // S^T double buffer: 2 x NH columns
   static constexpr int TMEM_O = 2 * NH;             // O^T: DVB x NH columns
   static constexpr uint32_t TMEM_COLS = ceil_pow2_cols(2 * NH + DVB * NH);
   static_assert(QT_BYTES % 1024 == 0, "Q^T buffers must keep 1024-byte alignment");
   static_assert(OFF_PT % 1024 == 0, "P^T alignment");
-  static_assert(RING % 2 == 0 && KSLOTS % 2 == 0 && VCH % 2 == 0, "V chunk pairs need even slots");
+  static_assert(GCH == 2 && RING % GCH == 0 && VG == DVB, "a V group is one 128-row O^T block");
   static_assert(NH % 16 == 0 && NH <= 256, "MMA N");
   static_assert(TMEM_COLS * CTAS <= 512, "TMEM");
   static_assert(SMEM_BYTES * CTAS <= 232448, "shared memory");
@@ -235,9 +243,9 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
   volatile int* abort_flag = flags + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 12);
   const uint32_t bar0 = sbase + T::OFF_BAR;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (T::RING + s); };
-  const uint32_t s_full = bar0 + 8u * (2 * T::RING);      // [2]
+  auto full_bar = [&](int g) { return bar0 + 8u * g; };
+  auto empty_bar = [&](int g) { return bar0 + 8u * (T::RING_G + g); };
+  const uint32_t s_full = bar0 + 8u * (2 * T::RING_G);    // [2]
   const uint32_t s_free = s_full + 16;                    // [2]
   const uint32_t p_full = s_free + 16;                    // [NPT]
   const uint32_t o_done = p_full + 8 * T::NPT;            // [NPT]
@@ -251,9 +259,9 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < T::RING; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int g = 0; g < T::RING_G; ++g) {
+      mbar_init(full_bar(g), 1);
+      mbar_init(empty_bar(g), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
@@ -303,36 +311,29 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const uint64_t pol = l2_policy_evict_first();
-      int slot = 0;
+      int grp = 0;
       uint32_t ph = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* map, int c0, int tok, int kvh, int b) {
+      // chunks [ch, ch + GCH) of key rows [tok, tok + 128) -> the next ring group
+      auto load = [&](const CUtensorMap* map, int ch, int tok, int kvh, int b) {
         if (!ok) return;
-        ok = mbar_wait(empty_bar(slot), ph ^ 1u, abort_flag, p.timeout_ns, 1);
+        ok = mbar_wait(empty_bar(grp), ph ^ 1u, abort_flag, p.timeout_ns, 1);
         if (!ok) return;
-        mbar_arrive_expect_tx(full_bar(slot), T::SLOT);
-        tma_load_4d(ring + slot * T::SLOT, map, full_bar(slot), c0, tok, kvh, b, pol);
-        if (++slot == T::RING) { slot = 0; ph ^= 1u; }
-      };
-      auto phantom = [&]() {
-        if (!ok) return;
-        ok = mbar_wait(empty_bar(slot), ph ^ 1u, abort_flag, p.timeout_ns, 2);
-        if (!ok) return;
-        mbar_arrive(full_bar(slot));
-        if (++slot == T::RING) { slot = 0; ph ^= 1u; }
+        mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
+        tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, tok, ch, kvh, b, pol);
+        if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
       };
       PieceWalker w = walker();
       int b, kvh, t0, n;
       int pv_tok = -1, pv_kvh = 0, pv_b = 0;  // tile whose V is still to be loaded
       auto load_v = [&]() {
-        for (int c = 0; c < T::VCH; ++c) load(&tmV, c * 64, pv_tok, pv_kvh, pv_b);
+        for (int c = 0; c < T::VCH; c += T::GCH) load(&tmV, c, pv_tok, pv_kvh, pv_b);
       };
       while (ok && w.next(b, kvh, t0, n)) {
         for (int i = 0; i < n && ok; ++i) {
           const int tok = (t0 + i) * T::TILE;
           if (i == 0 && pv_tok >= 0) load_v();  // finish the previous piece first
-          for (int c = 0; c < T::KCH; ++c) load(&tmK, c * 64, tok, kvh, b);
-          if (T::KSLOTS > T::KCH) phantom();
+          for (int c = 0; c < T::KCH; c += T::GCH) load(&tmK, c, tok, kvh, b);
           if (i > 0) load_v();
           pv_tok = tok;
           pv_kvh = kvh;
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       // one elected lane issues; waits are polled by the converged warp)
       constexpr uint32_t idS = umma_idesc(128, NH, BF16, false, false);
       constexpr uint32_t idO = umma_idesc(128, NH, BF16, true, true);
-      int slot = 0;
+      int grp = 0;
       uint32_t ph = 0;
       bool ok = true;
       auto pv = [&](int t, bool first_of_piece) {
@@ -377,27 +378,25 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
         // K step = 2*NH*16 bytes.
         const uint64_t bd0 = umma_sdesc(pt + pb * T::PT_BYTES, NH * 16, 128, SMEM_NOSWIZZLE);
         for (int i = 0; i < T::DVB; ++i) {
-          ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 5) &&
-               mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 5);
+          ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 5);
           if (!ok) return;
           tc_fence_after();
           if (elect_one()) {
             // A = V^T: MN-major, 128-byte swizzle; the two 64-row halves of
-            // the 128-row block sit one slot apart (LBO); 8-key groups are
-            // 1024 bytes apart (SBO); 16 keys per K step = 2048 bytes.
-            const uint64_t ad0 = umma_sdesc(ring + slot * T::SLOT, T::SLOT, 1024, SMEM_SW128);
+            // the 128-row block are the group's two chunks, one chunk apart
+            // (LBO); 8-key groups are 1024 bytes apart (SBO); 16 keys per K
+            // step = 2048 bytes.
+            const uint64_t ad0 = umma_sdesc(ring + grp * T::GBYTES, T::SLOT, 1024, SMEM_SW128);
             const uint32_t d = tmem + T::TMEM_O + i * NH;
             umma_ss(d, ad0, bd0, idO, first_of_piece ? 0u : 1u);
 #pragma unroll
             for (int ks = 1; ks < 8; ++ks)
               umma_ss(d, ad0 + (uint64_t)(ks * (2048 >> 4)), bd0 + (uint64_t)(ks * (2 * NH * 16 >> 4)),
                       idO, 1u);
-            umma_commit(empty_bar(slot));
-            umma_commit(empty_bar(slot + 1));
+            umma_commit(empty_bar(grp));
           }
           __syncwarp();
-          slot += 2;
-          if (slot == T::RING) { slot = 0; ph ^= 1u; }
+          if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
         }
         if (elect_one()) umma_commit(o_done + 8 * pb);
         __syncwarp();
@@ -417,19 +416,17 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
           if (j >= 2) ok = mbar_wait_warp(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 7);
           if (!ok) break;
           tc_fence_after();
-          // K chunks are consumed in pairs (two ring slots, eight MMAs per
-          // wait); with an odd chunk count the last pair's second slot is the
-          // producer's empty placeholder.
+          // K chunks arrive in ring groups of two (eight MMAs per wait); the
+          // zero-filled second chunk of an odd count's last group is skipped.
           const uint32_t qbase = qt + (k % T::NQ) * T::QT_BYTES;
           for (int c = 0; c < T::KCH && ok; c += 2) {
-            ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 8) &&
-                 mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 8);
+            ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 8);
             if (!ok) break;
             tc_fence_after();
             if (elect_one()) {
               // A = K tile, B = Q^T: both K-major, 128-byte swizzle, 8-row
               // groups 1024 bytes apart; 16 columns per K step = 32 bytes.
-              const uint64_t ad0 = umma_sdesc(ring + slot * T::SLOT, 16, 1024, SMEM_SW128);
+              const uint64_t ad0 = umma_sdesc(ring + grp * T::GBYTES, 16, 1024, SMEM_SW128);
               const uint64_t bd0 = umma_sdesc(qbase + c * T::QT_CHUNK, 16, 1024, SMEM_SW128);
               const uint32_t d = tmem + T::TMEM_S + sb * NH;
               umma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
@@ -441,12 +438,10 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) umma_ss(d, ad1 + 2 * ks, bd1 + 2 * ks, idS, 1u);
               }
-              umma_commit(empty_bar(slot));
-              umma_commit(empty_bar(slot + 1));
+              umma_commit(empty_bar(grp));
             }
             __syncwarp();
-            slot += 2;
-            if (slot == T::RING) { slot = 0; ph ^= 1u; }
+            if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
           }
           if (!ok) break;
           if (elect_one()) {

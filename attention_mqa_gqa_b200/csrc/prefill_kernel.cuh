@@ -83,6 +83,12 @@ struct PrefillTraits {
   static constexpr int NQ = (DK >= 512) ? 1 : 2;  // Q buffers
   static constexpr int RING = (DK >= 512) ? 4 : 6;
   static constexpr int SLOT = 16384;
+  // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
+  // copies of a single 16 KB chunk cap a CTA's stream well below what the
+  // tensor cores consume
+  static constexpr int GCH = 2;
+  static constexpr int GBYTES = GCH * SLOT;
+  static constexpr int RING_G = RING / GCH;
   static constexpr int Q_BYTES = QCH * SLOT;
   static constexpr int P_BYTES = 2 * SLOT;       // P: [128 x 128] as two [128 x 64] chunks
   static constexpr int OFF_Q = 0;
@@ -91,16 +97,17 @@ struct PrefillTraits {
   static constexpr int OFF_XCH = OFF_RING + RING * SLOT;     // float [2][128]: row-half exchange
   static constexpr int OFF_FLAGS = OFF_XCH + 2 * 128 * 4;     // abort, tmem base
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
-  // full[RING], empty[RING], q_full[NQ], q_free[NQ], s_full[2], s_free[2], p_full[NPBUF],
-  // o_done[NPBUF], o_free, drain
-  static constexpr int NBAR = 2 * RING + 2 * NQ + 6 + 2 * NPBUF;
+  // full[RING_G], empty[RING_G], q_full[NQ], q_free[NQ], s_full[2], s_free[2],
+  // p_full[NPBUF], o_done[NPBUF], o_free, drain
+  static constexpr int NBAR = 2 * RING_G + 2 * NQ + 6 + 2 * NPBUF;
   static constexpr int SOFTMAX_THREADS = 256;    // two threads per q row (64 keys each)
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int TMEM_S = 0;               // two S buffers, 128 columns each
   static constexpr int TMEM_O = 256;             // DVH columns
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(KCH % 2 == 0 && VCH % 2 == 0 && RING % 2 == 0, "V chunk pairs need even slots");
+  static_assert(KCH % GCH == 0 && VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
+                "chunks travel in pairs; a V pair is one 128-column block of O");
   static_assert(TMEM_O + DVH <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -122,9 +129,9 @@ __global__ void __launch_bounds__(64 + 256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 4);
   const uint32_t bar0 = sbase + T::OFF_BAR;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (T::RING + s); };
-  const uint32_t q_full = bar0 + 8u * (2 * T::RING);   // [NQ]
+  auto full_bar = [&](int g) { return bar0 + 8u * g; };
+  auto empty_bar = [&](int g) { return bar0 + 8u * (T::RING_G + g); };
+  const uint32_t q_full = bar0 + 8u * (2 * T::RING_G);  // [NQ]
   const uint32_t q_free = q_full + 8 * T::NQ;          // [NQ]
   const uint32_t s_full = q_free + 8 * T::NQ;          // [2]
   const uint32_t s_free = s_full + 16;                 // [2]
@@ -137,9 +144,9 @@ __global__ void __launch_bounds__(64 + 256, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < T::RING; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int g = 0; g < T::RING_G; ++g) {
+      mbar_init(full_bar(g), 1);
+      mbar_init(empty_bar(g), 1);
     }
     for (int i = 0; i < T::NQ; ++i) {
       mbar_init(q_full + 8 * i, 1);
@@ -172,32 +179,33 @@ __global__ void __launch_bounds__(64 + 256, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     const uint64_t pol_kv = l2_policy_evict_last();  // shared by the group's heads
-    int slot = 0;
+    int grp = 0;
     uint32_t ph = 0;
     bool ok = true;
-    auto load = [&](const CUtensorMap* map, int c0, int c1, int kvh, int b) {
+    // chunks [ch, ch + GCH) of key rows [row, row + 128) -> the next ring group
+    auto load = [&](const CUtensorMap* map, int ch, int row, int kvh, int b) {
       if (!ok) return;
-      ok = mbar_wait(empty_bar(slot), ph ^ 1u, abort_flag, p.timeout_ns, 21);
+      ok = mbar_wait(empty_bar(grp), ph ^ 1u, abort_flag, p.timeout_ns, 21);
       if (!ok) return;
-      mbar_arrive_expect_tx(full_bar(slot), T::SLOT);
-      tma_load_4d(ring + slot * T::SLOT, map, full_bar(slot), c0, c1, kvh, b, pol_kv);
-      if (++slot == T::RING) { slot = 0; ph ^= 1u; }
+      mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
+      tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, row, ch, kvh, b, pol_kv);
+      if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
     };
     bool have_prev = false;
-    int pv_tok = 0, pv_kvh = 0, pv_b = 0, pv_col = 0;  // tile whose V is still to load
+    int pv_tok = 0, pv_kvh = 0, pv_b = 0, pv_ch = 0;  // tile whose V is still to load
     auto load_v = [&]() {
-      for (int c = 0; c < T::VCH; ++c) load(&tmV, pv_col + c * 64, pv_tok, pv_kvh, pv_b);
+      for (int c = 0; c < T::VCH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
     };
     for (int L = blockIdx.x; L < p.n_items && ok; L += gridDim.x) {
       const PrefillItem it = prefill_item(p, L);
       for (int j = 0; j < it.ntiles && ok; ++j) {
         if (j == 0 && have_prev) load_v();  // finish the previous item first
-        for (int c = 0; c < T::KCH; ++c) load(&tmK, c * 64, j * T::KT, it.kvh, it.b);
+        for (int c = 0; c < T::KCH; c += T::GCH) load(&tmK, c, j * T::KT, it.kvh, it.b);
         if (j > 0) load_v();
         pv_tok = j * T::KT;
         pv_kvh = it.kvh;
         pv_b = it.b;
-        pv_col = it.part * DVH;
+        pv_ch = it.part * (DVH / 64);
         have_prev = true;
       }
     }
@@ -216,8 +224,8 @@ __global__ void __launch_bounds__(64 + 256, 1)
         ok = mbar_wait(q_free + 8 * qb, ((kq - T::NQ) / T::NQ) & 1, abort_flag, p.timeout_ns, 22);
       if (!ok) break;
       mbar_arrive_expect_tx(q_full + 8 * qb, T::Q_BYTES);
-      for (int c = 0; c < T::QCH; ++c)
-        tma_load_4d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, c * 64, it.q0,
+      for (int c = 0; c < T::QCH; c += T::GCH)
+        tma_load_5d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, 0, it.q0, c,
                     it.h, it.b, pol_q);
       ++kq;
     }
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
     // one elected lane issues; waits are polled by the converged warp)
     constexpr uint32_t idS = umma_idesc(128, 128, BF16, false, false);  // Q, K both K-major
     constexpr uint32_t idO = umma_idesc(128, 128, BF16, false, true);   // P K-major, V MN-major
-    int slot = 0;
+    int grp = 0;
     uint32_t ph = 0;
     bool ok = true;
     // PV(t): O += P(t) V(t); the first tile of item k > 0 first waits until
@@ -240,11 +248,10 @@ __global__ void __launch_bounds__(64 + 256, 1)
       tc_fence_after();
       const uint32_t abase = ps + pb * T::P_BYTES;
       for (int i = 0; i < T::VCH / 2; ++i) {
-        ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 25) &&
-             mbar_wait_warp(full_bar(slot + 1), ph, abort_flag, p.timeout_ns, 25);
+        ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 25);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t bbase = ring + slot * T::SLOT;
+        const uint32_t bbase = ring + grp * T::GBYTES;
         if (elect_one()) {
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
@@ -252,16 +259,14 @@ __global__ void __launch_bounds__(64 + 256, 1)
             const uint64_t ad =
                 umma_sdesc(abase + (ks >> 2) * T::SLOT + (ks & 3) * 32, 16, 1024, SMEM_SW128);
             // B = V: MN-major (d contiguous), 128-byte swizzle; the two 64-column
-            // halves are one slot apart (LBO), 8-key groups 1024 bytes (SBO).
+            // halves are the group's two chunks (LBO), 8-key groups 1024 bytes (SBO).
             const uint64_t bd = umma_sdesc(bbase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
             umma_ss(tmem + T::TMEM_O + i * 128, ad, bd, idO, (!first || ks > 0) ? 1u : 0u);
           }
-          umma_commit(empty_bar(slot));
-          umma_commit(empty_bar(slot + 1));
+          umma_commit(empty_bar(grp));
         }
         __syncwarp();
-        slot += 2;
-        if (slot == T::RING) { slot = 0; ph ^= 1u; }
+        if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
       }
       if (elect_one()) umma_commit(o_done + 8 * pb);
       __syncwarp();
@@ -282,23 +287,26 @@ __global__ void __launch_bounds__(64 + 256, 1)
         if (j >= 2) ok = mbar_wait_warp(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 27);
         if (!ok) break;
         tc_fence_after();
-        for (int c = 0; c < T::KCH && ok; ++c) {
-          ok = mbar_wait_warp(full_bar(slot), ph, abort_flag, p.timeout_ns, 28);
+        for (int c = 0; c < T::KCH && ok; c += T::GCH) {
+          ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 28);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t bbase = ring + slot * T::SLOT;
-          const uint32_t abase = qs + qb * T::Q_BYTES + c * T::SLOT;
           if (elect_one()) {
+            // A = Q chunks c, c+1; B = the group's two K chunks: both K-major,
+            // 128-byte swizzle, 8-row groups 1024 bytes apart, 32 bytes per K step
+            const uint64_t ad0 = umma_sdesc(qs + qb * T::Q_BYTES + c * T::SLOT, 16, 1024, SMEM_SW128);
+            const uint64_t bd0 = umma_sdesc(ring + grp * T::GBYTES, 16, 1024, SMEM_SW128);
+            const uint32_t d = tmem + T::TMEM_S + sb * 128;
+            umma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = umma_sdesc(abase + ks * 32, 16, 1024, SMEM_SW128);
-              const uint64_t bd = umma_sdesc(bbase + ks * 32, 16, 1024, SMEM_SW128);
-              umma_ss(tmem + T::TMEM_S + sb * 128, ad, bd, idS, (c > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 1; ks < 8; ++ks) {
+              const uint64_t off = (uint64_t)((ks >> 2) * (T::SLOT >> 4) + (ks & 3) * 2);
+              umma_ss(d, ad0 + off, bd0 + off, idS, 1u);
             }
-            umma_commit(empty_bar(slot));
+            umma_commit(empty_bar(grp));
           }
           __syncwarp();
-          if (++slot == T::RING) { slot = 0; ph ^= 1u; }
+          if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
         }
         if (!ok) break;
         if (elect_one()) {
