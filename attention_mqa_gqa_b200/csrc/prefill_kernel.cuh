@@ -11,7 +11,12 @@
 //
 //   S[128 x 128]   = Q_tile[128 x d_k] * K_tile^T            (tcgen05 -> TMEM)
 //   P = exp2(S*scale*log2e - m), row max m kept per thread (thread = row)
-//   O[128 x DVH]  += P[128 x 128] * V_tile[128 x DVH]        (tcgen05 -> TMEM)
+//   O[128 x DVH]  += P[128 x 128] * V_tile[128 x DVH]        (tcgen05, A from TMEM)
+//
+// P (bf16) is written back into the first 64 columns of its own S buffer
+// and read from there by the PV MMA, so it takes no shared memory and no
+// shared-memory bandwidth; the S buffer is reused for tile j + 2 once PV(j)
+// has completed.
 //
 // TMEM holds 512 fp32 columns per SM.  Two S buffers (256 columns) plus a
 // 128 x 512 fp32 O would need 768, so at d_v = 512 two work items share a
@@ -25,7 +30,7 @@
 // stream overlap the current item's last MMAs and epilogue.
 //
 // Warp roles (320 threads): warp 0 lane 0 streams K/V chunks through a ring
-// of 16 KB slots and lane 1 loads Q per item (TMA), warp 1 allocates TMEM
+// of 32 KB groups and lane 1 loads Q per item (TMA), warp 1 allocates TMEM
 // and issues UMMA, warps 2-9 run the softmax, rescale and epilogue: two
 // threads per q row (warps w and w+4 share a TMEM lane quarter), each owning
 // half of the row's keys and half of its output columns, exchanging the row
@@ -79,9 +84,8 @@ struct PrefillTraits {
   static constexpr int QCH = DK / 64;            // Q chunks ([128 x 64], 16 KB each)
   static constexpr int KCH = DK / 64;            // K chunks per key tile
   static constexpr int VCH = DVH / 64;           // V chunks per key tile (this item's columns)
-  static constexpr int NPBUF = (DK >= 512) ? 1 : 2;
   static constexpr int NQ = (DK >= 512) ? 1 : 2;  // Q buffers
-  static constexpr int RING = (DK >= 512) ? 4 : 6;
+  static constexpr int RING = (DK >= 512) ? 6 : 10;  // 16 KB chunk slots
   static constexpr int SLOT = 16384;
   // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
   // copies of a single 16 KB chunk cap a CTA's stream well below what the
@@ -90,20 +94,19 @@ struct PrefillTraits {
   static constexpr int GBYTES = GCH * SLOT;
   static constexpr int RING_G = RING / GCH;
   static constexpr int Q_BYTES = QCH * SLOT;
-  static constexpr int P_BYTES = 2 * SLOT;       // P: [128 x 128] as two [128 x 64] chunks
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = OFF_Q + NQ * Q_BYTES;
-  static constexpr int OFF_RING = OFF_P + NPBUF * P_BYTES;
+  static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_XCH = OFF_RING + RING * SLOT;     // float [2][128]: row-half exchange
   static constexpr int OFF_FLAGS = OFF_XCH + 2 * 128 * 4;     // abort, tmem base
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
-  // full[RING_G], empty[RING_G], q_full[NQ], q_free[NQ], s_full[2], s_free[2],
-  // p_full[NPBUF], o_done[NPBUF], o_free, drain
-  static constexpr int NBAR = 2 * RING_G + 2 * NQ + 6 + 2 * NPBUF;
+  // full[RING_G], empty[RING_G], q_full[NQ], q_free[NQ], s_full[2], p_full[2],
+  // o_done[2] (one of each per S/P buffer), o_free, drain
+  static constexpr int NBAR = 2 * RING_G + 2 * NQ + 8;
   static constexpr int SOFTMAX_THREADS = 256;    // two threads per q row (64 keys each)
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
-  static constexpr int TMEM_S = 0;               // two S buffers, 128 columns each
+  static constexpr int TMEM_S = 0;               // two S buffers, 128 columns each; P(j)
+                                                 // overwrites the first 64 of S(j)
   static constexpr int TMEM_O = 256;             // DVH columns
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(KCH % GCH == 0 && VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
@@ -123,7 +126,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
   const uint32_t sbase = smem_u32(smem);
 
   const uint32_t qs = sbase + T::OFF_Q;
-  const uint32_t ps = sbase + T::OFF_P;
   const uint32_t ring = sbase + T::OFF_RING;
   float* xch = reinterpret_cast<float*>(smem + T::OFF_XCH);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
@@ -133,11 +135,10 @@ __global__ void __launch_bounds__(64 + 256, 1)
   auto empty_bar = [&](int g) { return bar0 + 8u * (T::RING_G + g); };
   const uint32_t q_full = bar0 + 8u * (2 * T::RING_G);  // [NQ]
   const uint32_t q_free = q_full + 8 * T::NQ;          // [NQ]
-  const uint32_t s_full = q_free + 8 * T::NQ;          // [2]
-  const uint32_t s_free = s_full + 16;                 // [2]
-  const uint32_t p_full = s_free + 16;                 // [NPBUF]
-  const uint32_t o_done = p_full + 8 * T::NPBUF;       // [NPBUF]
-  const uint32_t o_free = o_done + 8 * T::NPBUF;
+  const uint32_t s_full = q_free + 8 * T::NQ;          // [2] S(j) in buffer j & 1
+  const uint32_t p_full = s_full + 16;                 // [2] P(j) written over S(j)
+  const uint32_t o_done = p_full + 16;                 // [2] PV(j) completed
+  const uint32_t o_free = o_done + 16;
   const uint32_t drain = o_free + 8;
 
   const int warp = threadIdx.x >> 5;
@@ -154,9 +155,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(s_free + 8 * i, T::SOFTMAX_THREADS);
-    }
-    for (int i = 0; i < T::NPBUF; ++i) {
       mbar_init(p_full + 8 * i, T::SOFTMAX_THREADS);
       mbar_init(o_done + 8 * i, 1);
     }
@@ -241,28 +239,27 @@ __global__ void __launch_bounds__(64 + 256, 1)
     // the epilogue of item k-1 has read O out of TMEM.
     auto pv = [&](int t, bool first, int k) {
       if (!ok) return;
-      const int pb = t % T::NPBUF;
-      ok = mbar_wait_warp(p_full + 8 * pb, (t / T::NPBUF) & 1, abort_flag, p.timeout_ns, 23);
+      const int pb = t & 1;
+      ok = mbar_wait_warp(p_full + 8 * pb, (t >> 1) & 1, abort_flag, p.timeout_ns, 23);
       if (ok && first && k > 0) ok = mbar_wait_warp(o_free, (k - 1) & 1, abort_flag, p.timeout_ns, 24);
       if (!ok) return;
       tc_fence_after();
-      const uint32_t abase = ps + pb * T::P_BYTES;
+      const uint32_t pcol = tmem + T::TMEM_S + pb * 128;  // P(t): 8 columns per 16 keys
       for (int i = 0; i < T::VCH / 2; ++i) {
         ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 25);
         if (!ok) return;
         tc_fence_after();
         const uint32_t bbase = ring + grp * T::GBYTES;
         if (elect_one()) {
+          // B = V: MN-major (d contiguous), 128-byte swizzle; the two 64-column
+          // halves are the group's two chunks (LBO), 8-key groups 1024 bytes
+          // (SBO), 16 keys per K step = 2048 bytes.  A = P(t) from TMEM.
+          const uint64_t bd0 = umma_sdesc(bbase, T::SLOT, 1024, SMEM_SW128);
+          const uint32_t d = tmem + T::TMEM_O + i * 128;
+          umma_ts(d, pcol, bd0, idO, first ? 0u : 1u);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            // A = P: K-major, 128-byte swizzle, keys 64*(ks/4) .. in chunk ks/4.
-            const uint64_t ad =
-                umma_sdesc(abase + (ks >> 2) * T::SLOT + (ks & 3) * 32, 16, 1024, SMEM_SW128);
-            // B = V: MN-major (d contiguous), 128-byte swizzle; the two 64-column
-            // halves are the group's two chunks (LBO), 8-key groups 1024 bytes (SBO).
-            const uint64_t bd = umma_sdesc(bbase + ks * 2048, T::SLOT, 1024, SMEM_SW128);
-            umma_ss(tmem + T::TMEM_O + i * 128, ad, bd, idO, (!first || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 1; ks < 8; ++ks)
+            umma_ts(d, pcol + ks * 8, bd0 + (uint64_t)(ks * (2048 >> 4)), idO, 1u);
           umma_commit(empty_bar(grp));
         }
         __syncwarp();
@@ -284,7 +281,8 @@ __global__ void __launch_bounds__(64 + 256, 1)
           ok = ok && mbar_wait_warp(q_full + 8 * qb, (kq / T::NQ) & 1, abort_flag, p.timeout_ns, 26);
           if (!ok) break;
         }
-        if (j >= 2) ok = mbar_wait_warp(s_free + 8 * sb, ((j >> 1) - 1) & 1, abort_flag, p.timeout_ns, 27);
+        // S buffer sb last held P(j - 2): PV(j - 2) must have completed
+        if (j >= 2) ok = mbar_wait_warp(o_done + 8 * sb, ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns, 27);
         if (!ok) break;
         tc_fence_after();
         for (int c = 0; c < T::KCH && ok; c += T::GCH) {
@@ -364,8 +362,6 @@ __global__ void __launch_bounds__(64 + 256, 1)
             for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
           }
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(s_free + 8 * sb);
 
           const int kb = i * T::KT + half * 64;
           // Keys at or past `lim` are invisible to this row; only tiles that
@@ -401,14 +397,10 @@ __global__ void __launch_bounds__(64 + 256, 1)
         const float m_new = need ? mx : m_used;
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
         const bool warp_need = __any_sync(0xffffffffu, need);
-        const int pb = j % T::NPBUF;
-        // P buffer pb was last read by PV(j - NPBUF); a failed wait ends the
-        // tile here and the pair leaves at the next pair_and
-        if (j >= T::NPBUF) ok = wait(o_done + 8 * pb, ((j - T::NPBUF) / T::NPBUF) & 1, 31);
-        if (!ok) continue;
+        // a failed wait ends the tile here and the pair leaves at the next pair_and
         if (warp_need && i > 0) {  // rescale this thread's O columns once PV(j-1) landed
           const int t = j - 1;
-          ok = wait(o_done + 8 * (t % T::NPBUF), (t / T::NPBUF) & 1, 32);
+          ok = wait(o_done + 8 * (t & 1), (t >> 1) & 1, 32);
           if (!ok) continue;
           tc_fence_after();
 #pragma unroll 1
@@ -426,33 +418,34 @@ __global__ void __launch_bounds__(64 + 256, 1)
         l *= alpha;
         m_used = m_new;
 
-        // P row half -> shared memory chunk `half` (K-major, 128-byte swizzle):
+        // P row half -> TMEM columns [32 * half, 32 * half + 32) of S buffer sb
+        // (two bf16 per column, keys in order; both halves of the row have read
+        // their S values before the pair barrier above):
         // p = exp2(s * scale * log2e - m), one FMA and one SFU op per key; a row
         // that has seen no visible key yet (m = -inf) writes zeros.
-        const uint32_t pbase = ps + pb * T::P_BYTES + half * T::SLOT;
         const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
         const bool none = m_used == -INFINITY;
         float lc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) lc[e] = 0.f;
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t u[4];
+        for (int h16 = 0; h16 < 2; ++h16) {
+          float u[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = c8 * 8 + 2 * e;
+          for (int e = 0; e < 16; ++e) {
+            const int c = h16 * 32 + 2 * e;
             const float p0 = none ? 0.f : ex2(fmaf(s[c], p.scale_log2, neg_m));
             const float p1 = none ? 0.f : ex2(fmaf(s[c + 1], p.scale_log2, neg_m));
-            u[e] = pack2(p0, p1, BF16);
-            lc[2 * e] += p0;
-            lc[2 * e + 1] += p1;
+            u[e] = __uint_as_float(pack2(p0, p1, BF16));
+            lc[(2 * e) & 7] += p0;
+            lc[(2 * e + 1) & 7] += p1;
           }
-          st_shared_v4(pbase + sw128_offset(row, c8 * 8), u[0], u[1], u[2], u[3]);
+          tmem_st16(tmem + lane_base + T::TMEM_S + sb * 128 + half * 32 + h16 * 16, u);
         }
         l += ((lc[0] + lc[1]) + (lc[2] + lc[3])) + ((lc[4] + lc[5]) + (lc[6] + lc[7]));
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full + 8 * pb);
+        mbar_arrive(p_full + 8 * sb);
       }
 
       // ------------------------------------------------------ epilogue
@@ -468,7 +461,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
       const float ltot = half == 0 ? lrow : xb[row];
       if (it.ntiles > 0) {
         const int t = j - 1;
-        ok = wait(o_done + 8 * (t % T::NPBUF), (t / T::NPBUF) & 1, 33);
+        ok = wait(o_done + 8 * (t & 1), (t >> 1) & 1, 33);
         if (!ok) continue;  // no pair barrier before the next item's first pair_and
         tc_fence_after();
       }
