@@ -15,6 +15,7 @@
 
 #include "../../include/attn_b200.h"
 #include "decode_kernel.cuh"
+#include "mla_pair_kernel.cuh"
 #include "prefill_kernel.cuh"
 
 namespace {
@@ -105,7 +106,10 @@ bool strides_ok(const attn_strides_t& s) {
 }
 
 // Resident decode CTAs per SM (must match DecodeTraits<...>::CTAS).
+// Decode CTAs resident per SM: two for d_k in {128, 512}; for MLA (576) one
+// CTA per SM, the SMs working in pairs (each pair one cluster of two CTAs).
 int decode_ctas_per_sm(int d_k) { return d_k == 576 ? 1 : 2; }
+bool decode_pairs(int d_k) { return d_k == 576; }
 
 bool shape_supported(int Sq, int d_k, int d_v) {
   if (Sq > 1) return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512);
@@ -136,16 +140,19 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
     return ATTN_OK;
   }
   pl->path = 1;
-  const int NH = d_k == 576 ? 64 : 16;
+  // heads per CTA (MLA: per CTA pair)
+  const int NH = d_k == 576 ? attn::MlaPairTraits::NH : 16;
   pl->heads_per_cta = NH;
   pl->head_blocks = (G + NH - 1) / NH;
   // One persistent wave: every SM runs decode_ctas_per_sm(d_k) CTAs; the
-  // key tiles are cut into equal ranges, one per CTA of each head block.
-  int ranges = num_sms * decode_ctas_per_sm(d_k) / pl->head_blocks;
+  // key tiles are cut into equal ranges, one per CTA (MLA: per pair) of
+  // each head block.
+  const int units_per_range = decode_pairs(d_k) ? 2 : 1;
+  int ranges = num_sms * decode_ctas_per_sm(d_k) / units_per_range / pl->head_blocks;
   if (ranges < 1) ranges = 1;
   pl->kv_ranges = ranges;
   pl->partials = (int64_t)ranges + (int64_t)B * Hkv;
-  pl->grid_ctas = (int64_t)ranges * pl->head_blocks;
+  pl->grid_ctas = (int64_t)ranges * pl->head_blocks * units_per_range;
   if (pl->grid_ctas > 0x7fffffffLL || (int64_t)B * Hq > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
   const size_t n = (size_t)pl->partials * G;
   pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float));
@@ -165,12 +172,44 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
                             const attn_plan_t& pl, cudaStream_t st, int phases) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
-  static_assert(Tr::CTAS == (DK == 576 ? 1 : 2), "decode_ctas_per_sm out of sync");
+  static_assert(Tr::CTAS == 2 && DK != 576, "decode_ctas_per_sm out of sync");
   if (phases & PHASE_PARTIAL) {
     auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
     set_smem(kern, Tr::SMEM_BYTES);
     kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  }
+  if (phases & PHASE_COMBINE) {
+    attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
+  }
+  return ATTN_OK;
+}
+
+template <bool BF16>
+attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const attn::DecodeParams& dp, const attn::CombineParams& cp,
+                              const attn_plan_t& pl, cudaStream_t st, int phases) {
+  using Tr = attn::MlaPairTraits;
+  if (phases & PHASE_PARTIAL) {
+    auto kern = attn::mla_pair_kernel<BF16>;
+    set_smem(kern, Tr::SMEM_BYTES);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
+    cfg.blockDim = dim3(Tr::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, dp) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ECUDA;
+    }
   }
   if (phases & PHASE_COMBINE) {
     attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
@@ -245,7 +284,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;
     if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
     CUtensorMap mq;
-    if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, (uint32_t)pl.heads_per_cta))
+    const uint32_t q_rows = decode_pairs(d_k) ? attn::MlaPairTraits::NHC : (uint32_t)pl.heads_per_cta;
+    if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, q_rows))
       return ATTN_ECUDA;
     attn::DecodeParams dp{};
     dp.skv = skv_per_seq;
@@ -275,14 +315,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     cp.G = G;
     cp.DV = d_v;
     cp.ranges = pl.kv_ranges;
+    cp.tile_shift = decode_pairs(d_k) ? attn::MlaPairTraits::TILE_SHIFT : 7;
     if (d_k == 128)
       return bf16 ? launch_decode<128, 128, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
                   : launch_decode<128, 128, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
     if (d_k == 512)
       return bf16 ? launch_decode<512, 512, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
                   : launch_decode<512, 512, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
-    return bf16 ? launch_decode<576, 512, 64, true>(mq, mk, mv, dp, cp, pl, st, phases)
-                : launch_decode<576, 512, 64, false>(mq, mk, mv, dp, cp, pl, st, phases);
+    return bf16 ? launch_mla_pair<true>(mq, mk, mv, dp, cp, pl, st, phases)
+                : launch_mla_pair<false>(mq, mk, mv, dp, cp, pl, st, phases);
   }
 
   if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;

@@ -55,7 +55,11 @@ constexpr uint32_t ceil_pow2_cols(uint32_t n) {
   return c;
 }
 
-__device__ __forceinline__ int key_tiles(int skv) { return (skv + 127) >> 7; }
+// Key tiles of a sequence: tiles of 2^shift keys (128 for one CTA, 256 for
+// a CTA pair).
+__device__ __forceinline__ int key_tiles(int skv, int shift) {
+  return (skv + (1 << shift) - 1) >> shift;
+}
 
 template <int DK, int DV, int NH>
 struct DecodeTraits {
@@ -145,12 +149,12 @@ __device__ __forceinline__ int transposed_head(int lane, int i) {
 // unit.  Every role of the CTA runs its own copy over the same range.
 struct PieceWalker {
   const int32_t* skv;
-  int B, Hkv;
+  int B, Hkv, shift;
   int b, kvh, off, remaining;
 
   __device__ bool next(int& pb, int& pkvh, int& tile0, int& ntiles) {
     if (remaining <= 0) return false;
-    const int tb = key_tiles(skv[b]);
+    const int tb = key_tiles(skv[b], shift);
     const int n = min(remaining, tb - off);
     pb = b;
     pkvh = kvh;
@@ -161,7 +165,7 @@ struct PieceWalker {
     if (remaining > 0) {
       if (++kvh == Hkv) {
         kvh = 0;
-        do { ++b; } while (b < B && key_tiles(skv[b]) == 0);
+        do { ++b; } while (b < B && key_tiles(skv[b], shift) == 0);
       }
     }
     return true;
@@ -172,15 +176,15 @@ struct PieceWalker {
 // all units (unit u = b * Hkv + kvh holds ceil(skv[b] / 128) tiles).  Called
 // by all threads of the CTA; leaves the range's first unit, tile offset and
 // length in sched[0..3] (length 0: no range r).
-__device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv, int R, int r,
-                                             long long* scan, int* sched) {
+__device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv, int shift, int R,
+                                             int r, long long* scan, int* sched) {
   const int tid = threadIdx.x;
   const int nt = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int c = (B + nt - 1) / nt;
   const int lo = min(B, tid * c), hi = min(B, lo + c);
   long long mine = 0;
-  for (int b = lo; b < hi; ++b) mine += key_tiles(skv[b]);
+  for (int b = lo; b < hi; ++b) mine += key_tiles(skv[b], shift);
   long long v = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -203,7 +207,7 @@ __device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv,
   if (tid == 0) sched[3] = (int)(x1 - x0);
   long long run = before + v - mine;  // tiles of sequences before `lo`
   for (int b = lo; b < hi; ++b) {
-    const int tb = key_tiles(skv[b]);
+    const int tb = key_tiles(skv[b], shift);
     const long long base = run * Hkv;
     if (tb > 0 && x0 < x1 && x0 >= base && x0 < base + (long long)tb * Hkv) {
       sched[0] = b;
@@ -287,7 +291,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
-  locate_range(p.skv, p.B, p.Hkv, p.ranges, rng, scan, sched);  // contains __syncthreads
+  locate_range(p.skv, p.B, p.Hkv, 7, p.ranges, rng, scan, sched);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
     w.skv = p.skv;
     w.B = p.B;
     w.Hkv = p.Hkv;
+    w.shift = 7;
     w.b = sched[0];
     w.kvh = sched[1];
     w.off = sched[2];
@@ -678,6 +683,7 @@ struct CombineParams {
   int64_t o_sb, o_sh;
   float* lse;  // [B, Hq] (Sq == 1) or NULL
   int B, Hq, Hkv, G, DV, ranges;
+  int tile_shift;  // log2 of the keys per tile the partial kernel used
 };
 
 // Largest range index r with floor(r * T / R) <= x (the range holding tile x).
@@ -707,7 +713,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   // tiles of the sequences before b, and of all sequences
   long long pre = 0, tot = 0;
   for (int bb = t; bb < p.B; bb += 128) {
-    const int tb = key_tiles(p.skv[bb]);
+    const int tb = key_tiles(p.skv[bb], p.tile_shift);
     tot += tb;
     if (bb < b) pre += tb;
   }
@@ -723,7 +729,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   __syncthreads();
   pre = (redl[0] + redl[1]) + (redl[2] + redl[3]);
   tot = (redl[4] + redl[5]) + (redl[6] + redl[7]);
-  const int tu = key_tiles(p.skv[b]);
+  const int tu = key_tiles(p.skv[b], p.tile_shift);
   const long long T = tot * p.Hkv;
   const long long Re = T < p.ranges ? T : p.ranges;  // ranges in use, none empty
   const long long u = (long long)b * p.Hkv + kvh;

@@ -45,11 +45,14 @@ def test_plan_decode_invariants(lib):
         pl = binding.plan(B, Hq, Hkv, 1, S, dk, dv, num_sms=148)
         G = Hq // Hkv
         assert pl["path"] == 1
-        assert pl["heads_per_cta"] == (64 if dk == 576 else 16)
+        # MLA runs on pairs of SMs (one cluster of two CTAs per key range)
+        # that together hold all 128 heads; the others 16 heads per CTA
+        assert pl["heads_per_cta"] == (128 if dk == 576 else 16)
         assert pl["head_blocks"] == -(-G // pl["heads_per_cta"])
+        ctas_per_range = 2 if dk == 576 else 1
         ctas_per_sm = 1 if dk == 576 else 2
-        assert pl["kv_ranges"] == max(1, 148 * ctas_per_sm // pl["head_blocks"])
-        assert pl["grid_ctas"] == pl["kv_ranges"] * pl["head_blocks"]
+        assert pl["kv_ranges"] == max(1, 148 * ctas_per_sm // ctas_per_range // pl["head_blocks"])
+        assert pl["grid_ctas"] == pl["kv_ranges"] * pl["head_blocks"] * ctas_per_range
         assert pl["partials"] == pl["kv_ranges"] + B * Hkv
         n = pl["partials"] * G
         r256 = lambda x: (x + 255) // 256 * 256
