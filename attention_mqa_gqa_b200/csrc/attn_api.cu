@@ -112,7 +112,10 @@ int decode_ctas_per_sm(int d_k) { return d_k == 576 ? 1 : 2; }
 bool decode_pairs(int d_k) { return d_k == 576; }
 
 bool shape_supported(int Sq, int d_k, int d_v) {
-  if (Sq > 1) return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512);
+  // prefill: GQA/MHA at 128, MQA at 512, and MLA prefill in its expanded
+  // (MHA) form: q_head_dim 192 = 128 + 64 rope columns, v_head_dim 128
+  if (Sq > 1)
+    return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512) || (d_k == 192 && d_v == 128);
   return (d_k == 128 && d_v == 128) || (d_k == 512 && d_v == 512) || (d_k == 576 && d_v == 512);
 }
 
@@ -351,6 +354,9 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   if (d_k == 128)
     return bf16 ? launch_prefill<128, 128, true>(mq, mk, mv, pp, pl, st)
                 : launch_prefill<128, 128, false>(mq, mk, mv, pp, pl, st);
+  if (d_k == 192)
+    return bf16 ? launch_prefill<192, 128, true>(mq, mk, mv, pp, pl, st)
+                : launch_prefill<192, 128, false>(mq, mk, mv, pp, pl, st);
   return bf16 ? launch_prefill<512, 256, true>(mq, mk, mv, pp, pl, st)
               : launch_prefill<512, 256, false>(mq, mk, mv, pp, pl, st);
 }

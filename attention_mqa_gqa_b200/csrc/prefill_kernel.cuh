@@ -81,11 +81,12 @@ template <int DK, int DVH>
 struct PrefillTraits {
   static constexpr int TILE = 128;               // q rows per item (MMA M)
   static constexpr int KT = 128;                 // keys per tile (MMA N of S)
-  static constexpr int QCH = DK / 64;            // Q chunks ([128 x 64], 16 KB each)
-  static constexpr int KCH = DK / 64;            // K chunks per key tile
+  static constexpr int KCH = DK / 64;            // 64-column chunks of a Q / K row
+  static constexpr int QCH = (KCH + 1) & ~1;     // chunk slots per Q row: pairs, the
+                                                 // last one zero-filled if KCH is odd
   static constexpr int VCH = DVH / 64;           // V chunks per key tile (this item's columns)
   static constexpr int NQ = (DK >= 512) ? 1 : 2;  // Q buffers
-  static constexpr int RING = (DK >= 512) ? 6 : 10;  // 16 KB chunk slots
+  static constexpr int RING = (DK >= 512 || QCH > 2) ? 6 : 10;  // 16 KB chunk slots
   static constexpr int SLOT = 16384;
   // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
   // copies of a single 16 KB chunk cap a CTA's stream well below what the
@@ -109,7 +110,7 @@ struct PrefillTraits {
                                                  // overwrites the first 64 of S(j)
   static constexpr int TMEM_O = 256;             // DVH columns
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(KCH % GCH == 0 && VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
+  static_assert(VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
                 "chunks travel in pairs; a V pair is one 128-column block of O");
   static_assert(TMEM_O + DVH <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -296,10 +297,12 @@ __global__ void __launch_bounds__(64 + 256, 1)
             const uint64_t bd0 = umma_sdesc(ring + grp * T::GBYTES, 16, 1024, SMEM_SW128);
             const uint32_t d = tmem + T::TMEM_S + sb * 128;
             umma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
+            // the second chunk of an odd count's last pair is padding: skipped
+            const int nks = c + 1 < T::KCH ? 8 : 4;
 #pragma unroll
             for (int ks = 1; ks < 8; ++ks) {
               const uint64_t off = (uint64_t)((ks >> 2) * (T::SLOT >> 4) + (ks & 3) * 2);
-              umma_ss(d, ad0 + off, bd0 + off, idS, 1u);
+              if (ks < nks) umma_ss(d, ad0 + off, bd0 + off, idS, 1u);
             }
             umma_commit(empty_bar(grp));
           }

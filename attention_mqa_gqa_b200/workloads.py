@@ -53,8 +53,9 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads: MQA d=512 prefill (tiny, fp16) and decode, MQA d=512
-# prefill, GQA 64/8 d=128 decode and prefill, absorbed-MLA decode.
+# The workloads: MQA d=512 prefill (tiny, fp16) and decode, MQA d=512
+# prefill, GQA 64/8 d=128 decode and prefill, absorbed-MLA decode, and
+# expanded-MLA prefill (d_k = 192, d_v = 128).
 WORKLOADS = {
     "mqa_prefill_tiny": Workload("mqa_prefill_tiny", 1, 16, 1, 128, 128, 128, 512, 512,
                                  torch.float16, True, 1 / math.sqrt(512), False, 0),
@@ -68,6 +69,10 @@ WORKLOADS = {
                             torch.bfloat16, True, 1 / math.sqrt(128), False, 3),
     "mla_decode": Workload("mla_decode", 64, 128, 1, 1, 4096, 16384, 576, 512,
                            torch.bfloat16, True, 1 / math.sqrt(192), True, 4),
+    # MLA prefill in the expanded (MHA) form: 128 heads, q/k head dim 192
+    # (128 nope + 64 rope columns, already rotated), v head dim 128
+    "mla_prefill": Workload("mla_prefill", 1, 128, 128, 4096, 4096, 4096, 192, 128,
+                            torch.bfloat16, True, 1 / math.sqrt(192), False, 5),
 }
 
 

@@ -115,6 +115,18 @@ def test_prefill_d512_noncausal_ragged():
     _case(2, 4, 1, 129, [129, 129], 512, 512, causal=False, seed=6)
 
 
+@pytest.mark.parametrize("Hq,Hkv,Sq,skv,causal", [(8, 8, 300, [300], True),
+                                                  (4, 2, 129, [200], True),
+                                                  (8, 8, 257, [257], False)])
+def test_prefill_mla_expanded(Hq, Hkv, Sq, skv, causal):
+    """MLA prefill in the expanded (MHA) form ("带你了解Attention" section 4.4:
+    prefill runs as ordinary attention on reconstructed K, V): q/k rows of
+    192 = 128 + 64 (rope) columns -- an odd number of 64-column chunks --
+    and v rows of 128, scale 1/sqrt(192)."""
+    _case(len(skv), Hq, Hkv, Sq, skv, 192, 128, causal=causal, seed=30 + Sq,
+          scale=1 / math.sqrt(192))
+
+
 def test_prefill_mqa_tiny_workload():
     """The MQA d=512 fp16 prefill workload (B=1, Hq=16, S=128) in full."""
     w = wl.WORKLOADS["mqa_prefill_tiny"]
@@ -167,6 +179,6 @@ def _sampled(name, n_pairs=12, n_rows=48, seed=0):
 
 
 @pytest.mark.parametrize("name", ["mqa_decode", "gqa_decode", "mla_decode", "mqa_prefill",
-                                  "gqa_prefill"])
+                                  "gqa_prefill", "mla_prefill"])
 def test_full_workload_sampled(name):
     _sampled(name)

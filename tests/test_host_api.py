@@ -120,6 +120,9 @@ def test_plan_prefill(lib):
     assert pl["dv_parts"] == 1 and pl["grid_ctas"] == 148
     pl = binding.plan(1, 2, 1, 100, 100, 128, 128, num_sms=148)
     assert pl["grid_ctas"] == 2  # fewer work items than SMs
+    # expanded MLA prefill: q/k 192 wide, v 128 wide, one d_v part
+    pl = binding.plan(1, 128, 128, 4096, 4096, 192, 128, num_sms=148)
+    assert pl["path"] == 0 and pl["dv_parts"] == 1 and pl["grid_ctas"] == 148
 
 
 @pytest.mark.parametrize("args,code", [
@@ -128,6 +131,7 @@ def test_plan_prefill(lib):
     ((1, 16, 1, 1, 0, 512, 512), binding.ATTN_EINVAL),         # no keys at all
     ((1, 16, 1, 1, 100, 256, 256), binding.ATTN_EUNSUPPORTED),
     ((1, 16, 1, 4, 100, 576, 512), binding.ATTN_EUNSUPPORTED),  # MLA shape is decode-only
+    ((1, 16, 16, 1, 100, 192, 128), binding.ATTN_EUNSUPPORTED),  # expanded MLA: prefill only
     ((1, 16, 1, 1, 100, 512, 128), binding.ATTN_EUNSUPPORTED),
 ])
 def test_plan_rejects(lib, args, code):
