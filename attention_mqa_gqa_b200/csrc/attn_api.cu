@@ -72,6 +72,27 @@ bool make_chunk_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_
 
 // 3-D map over q [B, Hq, 1, D] seen as rows (head) of D columns: box = 64
 // columns x `rows` heads, 128-byte swizzle (the decode kernel's Q^T chunks).
+// 4-D map over q [B, Hq, Sq, D]: box = 64 columns x Sq queries x
+// `heads` heads, 128-byte swizzle; lands as Q^T rows head * Sq + query (the
+// decode kernel's columns).
+bool make_q_cols_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t Sq,
+                     uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb, uint32_t heads) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  if (Sq == 1) ss = (int64_t)D;
+  if (H == 1) sh = ss * (int64_t)Sq;
+  if (B == 1) sb = sh * (int64_t)H;
+  cuuint64_t dims[4] = {D, Sq, H, B};
+  cuuint64_t strides[3] = {(cuuint64_t)ss * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)Sq, heads, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_q_rows_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t H,
                      uint64_t B, int64_t sh, int64_t sb, uint32_t rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -121,6 +142,19 @@ bool shape_supported(int Sq, int d_k, int d_v) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Columns (head x query) per decode CTA for d_k in {128, 512}.
+constexpr int kDecodeCols = 16;
+
+// A few queries per sequence against a long cache (extend, speculative
+// decoding) run through the split-KV decode kernel with the G heads x Sq
+// queries of a kv head as MMA columns: Sq a power of two dividing the
+// columns of a CTA.  MLA decode (576) takes Sq == 1 only; longer query
+// blocks go to the prefill kernel.
+bool decode_path(int Sq, int d_k) {
+  if (Sq == 1) return true;
+  return (d_k == 128 || d_k == 512) && Sq <= kDecodeCols && (Sq & (Sq - 1)) == 0;
+}
+
 attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, int d_v,
                         attn_dtype_t dtype, int num_sms, attn_plan_t* pl) {
   if (!pl) return ATTN_EINVAL;
@@ -132,7 +166,7 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
   if (!shape_supported(Sq, d_k, d_v)) return ATTN_EUNSUPPORTED;
   if (num_sms <= 0) num_sms = device_sm_count();
   const int G = Hq / Hkv;
-  if (Sq > 1) {
+  if (!decode_path(Sq, d_k)) {
     pl->path = 0;
     pl->dv_parts = d_v / (d_v >= 512 ? 256 : 128);
     const int64_t n_qt = (Sq + 127) / 128;
@@ -143,10 +177,11 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
     return ATTN_OK;
   }
   pl->path = 1;
-  // heads per CTA (MLA: per CTA pair)
-  const int NH = d_k == 576 ? attn::MlaPairTraits::NH : 16;
+  // columns (head x query) per CTA (MLA: heads per CTA pair)
+  const int NH = d_k == 576 ? attn::MlaPairTraits::NH : kDecodeCols;
+  const int GC = G * Sq;
   pl->heads_per_cta = NH;
-  pl->head_blocks = (G + NH - 1) / NH;
+  pl->head_blocks = (GC + NH - 1) / NH;
   // One persistent wave: every SM runs decode_ctas_per_sm(d_k) CTAs; the
   // key tiles are cut into equal ranges, one per CTA (MLA: per pair) of
   // each head block.
@@ -156,8 +191,9 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
   pl->kv_ranges = ranges;
   pl->partials = (int64_t)ranges + (int64_t)B * Hkv;
   pl->grid_ctas = (int64_t)ranges * pl->head_blocks * units_per_range;
-  if (pl->grid_ctas > 0x7fffffffLL || (int64_t)B * Hq > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
-  const size_t n = (size_t)pl->partials * G;
+  if (pl->grid_ctas > 0x7fffffffLL || (int64_t)B * Hq * Sq > 0x7fffffffLL)
+    return ATTN_EUNSUPPORTED;
+  const size_t n = (size_t)pl->partials * GC;
   pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float));
   return ATTN_OK;
 }
@@ -183,7 +219,7 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   if (phases & PHASE_COMBINE) {
-    attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
+    attn::combine_kernel<BF16><<<dp.B * dp.Hq * dp.Sq, 128, 0, st>>>(cp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   return ATTN_OK;
@@ -215,7 +251,7 @@ attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, cons
     }
   }
   if (phases & PHASE_COMBINE) {
-    attn::combine_kernel<BF16><<<dp.B * dp.Hq, 128, 0, st>>>(cp);
+    attn::combine_kernel<BF16><<<dp.B * dp.Hq * dp.Sq, 128, 0, st>>>(cp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   return ATTN_OK;
@@ -287,12 +323,16 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;
     if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
     CUtensorMap mq;
-    const uint32_t q_rows = decode_pairs(d_k) ? attn::MlaPairTraits::NHC : (uint32_t)pl.heads_per_cta;
-    if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, q_rows))
+    if (decode_pairs(d_k)) {
+      if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, attn::MlaPairTraits::NHC))
+        return ATTN_ECUDA;
+    } else if (!make_q_cols_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b,
+                                (uint32_t)(kDecodeCols / Sq))) {
       return ATTN_ECUDA;
+    }
     attn::DecodeParams dp{};
     dp.skv = skv_per_seq;
-    const size_t n = (size_t)pl.partials * G;
+    const size_t n = (size_t)pl.partials * G * Sq;
     dp.ws_o = reinterpret_cast<float*>(workspace);
     dp.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                          align256(n * d_v * sizeof(float)));
@@ -300,6 +340,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     dp.Hq = Hq;
     dp.Hkv = Hkv;
     dp.G = G;
+    dp.Sq = Sq;
+    dp.causal = causal;
     dp.ranges = pl.kv_ranges;
     dp.head_blocks = pl.head_blocks;
     dp.scale_log2 = scale_log2;
@@ -311,11 +353,13 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     cp.out = out;
     cp.o_sb = so.b;
     cp.o_sh = so.h;
+    cp.o_ss = so.s;
     cp.lse = lse;
     cp.B = B;
     cp.Hq = Hq;
     cp.Hkv = Hkv;
     cp.G = G;
+    cp.Sq = Sq;
     cp.DV = d_v;
     cp.ranges = pl.kv_ranges;
     cp.tile_shift = decode_pairs(d_k) ? attn::MlaPairTraits::TILE_SHIFT : 7;

@@ -41,9 +41,11 @@ namespace attn {
 
 struct DecodeParams {
   const int32_t* skv;    // [B] keys per sequence (device)
-  float* ws_o;           // [ranges + B*Hkv][G][d_v] normalised partial outputs
-  float* ws_lse;         // [ranges + B*Hkv][G] partial LSE (natural log)
+  float* ws_o;           // [ranges + B*Hkv][G*Sq][d_v] normalised partial outputs
+  float* ws_lse;         // [ranges + B*Hkv][G*Sq] partial LSE (natural log)
   int B, Hq, Hkv, G;
+  int Sq;                // queries per sequence (1, or a few for extend / speculative decode)
+  int causal;            // Sq > 1: query i sees keys j <= i + skv[b] - Sq
   int ranges, head_blocks;
   float scale_log2;      // scale * log2(e)
   uint64_t timeout_ns;
@@ -232,7 +234,10 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
 
   const int hb = blockIdx.x % p.head_blocks;     // head block of the group
   const int rng = blockIdx.x / p.head_blocks;    // key range
-  const int nvalid = min(NH, p.G - hb * NH);     // real heads among the NH rows
+  // The N dimension holds "columns" (head g of the group, query i), column
+  // g * Sq + i; NH columns per CTA (NH / Sq heads x Sq queries).
+  const int GC = p.G * p.Sq;                     // columns per kv head
+  const int nvalid = min(NH, GC - hb * NH);      // real columns among the NH rows
 
   const uint32_t ring = sbase + T::OFF_RING;
   const uint32_t qt = sbase + T::OFF_QT;
@@ -359,9 +364,10 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
           ok = mbar_wait(q_free + 8 * qb, ((k - T::NQ) / T::NQ) & 1, abort_flag, p.timeout_ns, 3);
         if (!ok) break;
         mbar_arrive_expect_tx(q_full + 8 * qb, T::QT_BYTES);
+        // box: 64 columns x Sq queries x NH/Sq heads -> Q^T rows g * Sq + i
         for (int c = 0; c < T::KCH; ++c)
-          tma_load_3d(qt + qb * T::QT_BYTES + c * T::QT_CHUNK, &tmQ, q_full + 8 * qb, c * 64,
-                      kvh * p.G + hb * NH, b, pol);
+          tma_load_4d(qt + qb * T::QT_BYTES + c * T::QT_CHUNK, &tmQ, q_full + 8 * qb, c * 64, 0,
+                      kvh * p.G + hb * (NH / p.Sq), b, pol);
         ++k;
       }
     } else if (warp == 1) {
@@ -500,7 +506,14 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
           ok = wait(s_full + 8 * sb, (j >> 1) & 1, 11);
           if (!ok) break;
           tc_fence_after();
-          const bool valid = (t0 + i) * T::TILE + row < skv_b;
+          // Column c holds query qi = c % Sq (Sq a power of two), which sees
+          // keys <= skv_b - Sq + qi under the causal mask (bottom-right
+          // alignment) and keys < skv_b otherwise; with kq = key - (skv_b - Sq)
+          // the causal test is kq <= qi.
+          const int key = (t0 + i) * T::TILE + row;
+          const int kq = key - (skv_b - p.Sq);
+          const bool in_seq = key < skv_b;
+          const int sq_mask = p.Sq - 1;
           // This thread's HH scores of its key (scaled to log2 units, masked),
           // read from TMEM twice: for the maxima and again for the weights,
           // so that only one HH-wide array is live at a time.
@@ -508,7 +521,10 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
             tmem_ld<HH>(tmem + lane_base + T::TMEM_S + sb * NH + h0l, x);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < HH; ++e) x[e] = valid ? x[e] * p.scale_log2 : -INFINITY;
+            for (int e = 0; e < HH; ++e) {
+              const bool vis = p.causal ? kq <= ((h0l + e) & sq_mask) : in_seq;
+              x[e] = vis ? x[e] * p.scale_log2 : -INFINITY;
+            }
           };
 
           // per-head maximum over the tile's 128 keys
@@ -631,7 +647,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
             const float L = (rbuf[st] + rbuf[NH + st]) + (rbuf[2 * NH + st] + rbuf[3 * NH + st]);
             l_sm[st] = L;
             if (st < nvalid)
-              p.ws_lse[slot_id * p.G + hb * NH + st] =
+              p.ws_lse[slot_id * GC + hb * NH + st] =
                   L > 0.f ? (m_sm[st] + __log2f(L)) * 0.69314718055994531f : -INFINITY;
             m_sm[st] = -INFINITY;  // the next piece starts afresh
             mbar_arrive(stat_ready + 8 * rb);
@@ -650,7 +666,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
               const int h = h0l + c;
               if (h < nvalid) {
                 const float L = l_sm[h];
-                p.ws_o[(slot_id * p.G + hb * NH + h) * DV + dd] = L > 0.f ? o[c] / L : 0.f;
+                p.ws_o[(slot_id * GC + hb * NH + h) * DV + dd] = L > 0.f ? o[c] / L : 0.f;
               }
             }
           }
@@ -672,7 +688,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
 
 // ---------------------------------------------------------------- combine
 //
-// out[b,h,0,:] = sum_s exp(lse_s - L) o_s,  L = log sum_s exp(lse_s), over
+// out[b,h,i,:] = sum_s exp(lse_s - L) o_s,  L = log sum_s exp(lse_s), over
 // the pieces of unit (b, h / G), in range order (no atomics, so the result
 // is bitwise reproducible: "GQA和MLA详解" section 4 on reduction order).
 struct CombineParams {
@@ -681,8 +697,10 @@ struct CombineParams {
   const int32_t* skv;
   void* out;
   int64_t o_sb, o_sh;
-  float* lse;  // [B, Hq] (Sq == 1) or NULL
+  int64_t o_ss;
+  float* lse;  // [B, Hq, Sq] or NULL
   int B, Hq, Hkv, G, DV, ranges;
+  int Sq;          // queries per sequence (columns per head)
   int tile_shift;  // log2 of the keys per tile the partial kernel used
 };
 
@@ -693,7 +711,7 @@ __device__ __forceinline__ long long range_of(long long x, long long T, long lon
 
 template <bool BF16>
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
-  // One block per (b, h).  The piece weights w_s = exp(lse_s - L) are
+  // One block per (b, h, query i).  The piece weights w_s = exp(lse_s - L) are
   // computed once into shared memory; each thread then owns 4 consecutive
   // d_v columns (float4) of one piece-group g and accumulates its pieces
   // s = g, g + NG, ... in order; the NG group sums are added in group order.
@@ -702,11 +720,14 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   __shared__ float red[4];
   __shared__ long long redl[8];
   __shared__ float4 part[128];
-  const int bh = blockIdx.x;
+  const int bhi = blockIdx.x;  // (b, h, query i)
+  const int qi = bhi % p.Sq;
+  const int bh = bhi / p.Sq;
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int kvh = h / p.G;
-  const int gh = h % p.G;
+  const int gh = (h % p.G) * p.Sq + qi;  // column within the kv head's G * Sq
+  const int GC = p.G * p.Sq;
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
 
@@ -742,7 +763,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
     n = min(n, MAXS);
   }
   // piece s of this unit lives in workspace slot (r_lo + s) + u
-  auto slot = [&](int s) { return (r_lo + s + u) * p.G + gh; };
+  auto slot = [&](int s) { return (r_lo + s + u) * GC + gh; };
 
   float mx = -INFINITY;
   for (int s = t; s < n; s += 128) mx = fmaxf(mx, p.ws_lse[slot(s)]);
@@ -804,10 +825,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   }
   if (g == 0) {
     uint8_t* outp =
-        reinterpret_cast<uint8_t*>(p.out) + ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + d4 * 4) * 2;
+        reinterpret_cast<uint8_t*>(p.out) +
+        ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)qi * p.o_ss + d4 * 4) * 2;
     *reinterpret_cast<uint2*>(outp) = make_uint2(pack2(acc.x, acc.y, BF16), pack2(acc.z, acc.w, BF16));
   }
-  if (t == 0 && p.lse) p.lse[bh] = L;
+  if (t == 0 && p.lse) p.lse[bhi] = L;
 }
 
 }  // namespace attn

@@ -47,7 +47,13 @@ class Workload:
 
     @property
     def is_decode(self) -> bool:
-        return self.Sq == 1
+        """Runs on the split-KV decode path and is bound by reading the KV
+        cache: one query per sequence, or a few (a power of two up to 16 at
+        head dim 128 or 512: extend / speculative-decoding verification)."""
+        if self.Sq == 1:
+            return True
+        return (self.d_k in (128, 512) and self.d_k == self.d_v and self.Sq <= 16
+                and self.Sq & (self.Sq - 1) == 0)
 
     def scaled(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -69,6 +75,9 @@ WORKLOADS = {
                             torch.bfloat16, True, 1 / math.sqrt(128), False, 3),
     "mla_decode": Workload("mla_decode", 64, 128, 1, 1, 4096, 16384, 576, 512,
                            torch.bfloat16, True, 1 / math.sqrt(192), True, 4),
+    # speculative-decoding verify step: 4 queries per sequence against the cache
+    "gqa_extend": Workload("gqa_extend", 64, 64, 8, 4, 4096, 4096, 128, 128,
+                           torch.bfloat16, True, 1 / math.sqrt(128), False, 6),
     # MLA prefill in the expanded (MHA) form: 128 heads, q/k head dim 192
     # (128 nope + 64 rope columns, already rotated), v head dim 128
     "mla_prefill": Workload("mla_prefill", 1, 128, 128, 4096, 4096, 4096, 192, 128,

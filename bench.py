@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 from attention_mqa_gqa_b200 import workloads as wl  # noqa: E402
 
 KERNEL_SOURCES = ["attention_mqa_gqa_b200/csrc/sm100.cuh", "attention_mqa_gqa_b200/csrc/decode_kernel.cuh",
+                  "attention_mqa_gqa_b200/csrc/mla_pair_kernel.cuh",
                   "attention_mqa_gqa_b200/csrc/prefill_kernel.cuh", "attention_mqa_gqa_b200/csrc/attn_api.cu"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -514,7 +515,7 @@ def main():
     value = work_all * steps / (max_ms * 1e-3) / scale_div
     metric, unit, hib = metric_of(w)
     long_run = total_ms > 1000.0
-    kname = "decode_split_kernel" if g.decode else "prefill_kernel"
+    kname = ("mla_pair_kernel" if w.mla else "decode_split_kernel") if g.decode else "prefill_kernel"
     roof = roofline(w, inp["skv"], k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
     roof["kernel"] = kname
     roof["kernel_ms"] = round(k_ms, 5)

@@ -38,9 +38,13 @@
  *   device-side waits that exceed their time limit set a device error word
  *   read by attn_last_device_error().
  *
- * Supported shapes: (d_k, d_v) in {(128,128), (512,512)} for prefill
- * (Sq > 1) and decode (Sq == 1); (576, 512) for decode.  Element type bf16
- * or fp16.  Anything else returns ATTN_EUNSUPPORTED; there is no fallback.
+ * Supported shapes: (d_k, d_v) in {(128,128), (512,512)} for any Sq;
+ * (576, 512) -- absorbed MLA over [c_kv | k_pe] rows -- for decode (Sq == 1);
+ * (192, 128) -- MLA prefill in its expanded (MHA) form -- for Sq > 1.
+ * Sq == 1, and Sq in {2, 4, 8, 16} at d_k in {128, 512} (extend / speculative
+ * decoding against a cache), take the split-KV decode path; other Sq > 1 the
+ * prefill kernel.  Element type bf16 or fp16.  Anything else returns
+ * ATTN_EUNSUPPORTED; there is no fallback.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -71,8 +75,10 @@ typedef struct {
 /* What attn_fwd will launch for a problem (host-side plan, no GPU needed). */
 typedef struct {
   int path;            /* 0 = prefill kernel, 1 = split-KV decode + combine      */
-  int heads_per_cta;   /* decode: query heads packed into one CTA (MMA N)       */
-  int head_blocks;     /* decode: CTAs per key range along the group's heads    */
+  int heads_per_cta;   /* decode: (query head x query) columns packed into one
+                          CTA's MMA N (MLA: heads per pair of CTAs)              */
+  int head_blocks;     /* decode: CTAs per key range along the group's G * Sq
+                          columns                                                */
   int kv_ranges;       /* decode: equal ranges the concatenated key tiles of all
                           (sequence, kv head) pairs are cut into, one persistent
                           CTA per range and head block                           */
@@ -94,8 +100,8 @@ attn_status_t attn_plan(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
 
 /*
  * Workspace bytes attn_fwd needs for this problem on the current device
- * (0 for prefill).  Decode stores partial outputs (fp32 [partials, G, d_v])
- * and partial LSEs (fp32 [partials, G]) there, one slot per piece of a
+ * (0 for prefill).  Decode stores partial outputs (fp32 [partials, G * Sq,
+ * d_v]) and partial LSEs (fp32 [partials, G * Sq]) there, one slot per piece of a
  * (sequence, kv head) pair that falls in one key range.  Returns 0 for
  * arguments attn_plan rejects.
  */
@@ -123,18 +129,18 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
                        void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
- * The two steps attn_fwd enqueues for a decode problem (Sq == 1), callable
+ * The two steps attn_fwd enqueues for a decode-path problem (plan path 1), callable
  * separately with attn_fwd's arguments (for timing each kernel, or for
  * overlapping the merge with other work):
  *   attn_decode_partial  -- one persistent CTA per key range and head block
  *                           attends over each piece of a (sequence, kv head)
  *                           pair in its range and writes a normalised partial
  *                           output and its LSE into the workspace;
- *   attn_decode_combine  -- merges the pieces of each (b, h) in range order:
+ *   attn_decode_combine  -- merges the pieces of each (b, h, query) in range order:
  *                           L = ln sum_s exp(lse_s), out = sum_s exp(lse_s - L) o_s
  *                           ("GQA和MLA详解" section 4: a fixed reduction order keeps
  *                           the result bitwise reproducible).
- * Same validation and errors as attn_fwd; ATTN_EINVAL when Sq > 1.  The
+ * Same validation and errors as attn_fwd; ATTN_EINVAL for prefill-path problems.  The
  * combine step reads what the partial step wrote into the same workspace.
  */
 attn_status_t attn_decode_partial(const void* q, const void* k, const void* v, void* out,

@@ -58,6 +58,20 @@ def test_decode_mla(Hq, skv):
     _case(len(skv), Hq, 1, 1, skv, 576, 512, mla=True, seed=11, scale=1 / math.sqrt(192))
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,skv,dk,causal", [
+    (3, 16, 2, 4, [1000, 3, 129], 128, True),    # skv < Sq: early queries see nothing
+    (2, 16, 2, 2, [700, 2], 128, True),
+    (2, 16, 2, 8, [4097, 300], 128, True),
+    (2, 16, 1, 4, [2000, 5], 512, True),
+    (2, 16, 2, 4, [777, 1], 128, False),
+    (2, 4, 4, 16, [1500, 20], 128, True),        # G = 1: 16 queries of one head per CTA
+])
+def test_decode_extend(B, Hq, Hkv, Sq, skv, dk, causal):
+    """Sq > 1 queries against a cache (extend / speculative decoding) on the
+    split-KV decode path, bottom-right causal alignment."""
+    _case(B, Hq, Hkv, Sq, skv, dk, dk, causal=causal, seed=40 + Sq)
+
+
 def test_decode_fp16():
     _case(2, 16, 1, 1, [333, 1000], 512, 512, dtype=torch.float16, seed=3)
 
@@ -171,7 +185,9 @@ def _sampled(name, n_pairs=12, n_rows=48, seed=0):
     else:
         rows = [(int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.Sq)))
                 for _ in range(n_rows)]
-        rows += [(0, 0, 0), (w.B - 1, w.Hq - 1, w.Sq - 1), (0, w.Hq - 1, 127), (0, 1, 128)]
+        rows += [(0, 0, 0), (w.B - 1, w.Hq - 1, w.Sq - 1)]
+        if w.Sq > 128:  # the rows on both sides of the first q-tile boundary
+            rows += [(0, w.Hq - 1, 127), (0, 1, 128)]
         ref_o, ref_l = npo.attention_rows(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(),
                                           w.scale, w.causal, rows)
         for r, (b, h, i) in enumerate(rows):
@@ -179,6 +195,6 @@ def _sampled(name, n_pairs=12, n_rows=48, seed=0):
 
 
 @pytest.mark.parametrize("name", ["mqa_decode", "gqa_decode", "mla_decode", "mqa_prefill",
-                                  "gqa_prefill", "mla_prefill"])
+                                  "gqa_prefill", "mla_prefill", "gqa_extend"])
 def test_full_workload_sampled(name):
     _sampled(name)

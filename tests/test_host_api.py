@@ -112,6 +112,21 @@ def test_schedule_slots_unique_and_cover():
             assert [x[0] for x in lst] == list(range(lst[0][0], lst[-1][0] + 1))
 
 
+def test_plan_extend_takes_decode_path(lib):
+    """A few queries against a long cache run as decode with G * Sq columns."""
+    for (Hq, Hkv, Sq, dk) in [(64, 8, 4, 128), (16, 1, 8, 512), (4, 4, 16, 128), (16, 2, 2, 512)]:
+        pl = binding.plan(5, Hq, Hkv, Sq, 4096, dk, dk, num_sms=148)
+        G = Hq // Hkv
+        assert pl["path"] == 1 and pl["heads_per_cta"] == 16
+        assert pl["head_blocks"] == -(-G * Sq // 16)
+        n = pl["partials"] * G * Sq
+        r256 = lambda x: (x + 255) // 256 * 256
+        assert pl["workspace_bytes"] == r256(n * dk * 4) + r256(n * 4)
+    for Sq in (3, 32, 100):  # not a power of two, or too many columns
+        assert binding.plan(5, 64, 8, Sq, 4096, 128, 128, num_sms=148)["path"] == 0
+    assert binding.plan(5, 128, 128, 4, 4096, 192, 128, num_sms=148)["path"] == 0
+
+
 def test_plan_prefill(lib):
     pl = binding.plan(2, 16, 1, 4096, 4096, 512, 512, num_sms=148)
     assert pl["path"] == 0 and pl["dv_parts"] == 2 and pl["workspace_bytes"] == 0
