@@ -200,13 +200,16 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
       // ------------------------------------------------ producer: K/V groups
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const uint64_t pol = l2_policy_evict_first();
+      // K rows stay in L2 until the pair reads their first 512 columns again
+      // as V (a tile later); that V read is their last use.
+      const uint64_t pol_k = l2_policy_evict_normal();
+      const uint64_t pol_v = l2_policy_evict_first();
       int grp = 0;
       uint32_t ph = 0;
       bool ok = true;
       // two chunks starting at `ch` of rows [row, row + 128); the bytes of
       // both CTAs' copies into group `grp` are counted on CTA 0's barrier
-      auto load = [&](const CUtensorMap* map, int ch, int row, int kvh, int b) {
+      auto load = [&](const CUtensorMap* map, int ch, int row, int kvh, int b, uint64_t pol) {
         if (!ok) return;
         ok = mbar_wait_cluster(empty_bar(grp), ph ^ 1u, abort_flag, p.timeout_ns, 41);
         if (!ok) return;
@@ -221,13 +224,14 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
       // V block m of this CTA = chunks 4m + 2cr, +1, for the tile's 256 keys
       auto load_v = [&]() {
         for (int m = 0; m < 2; ++m)
-          for (int h = 0; h < 2; ++h) load(&tmV, 4 * m + 2 * (int)cr, pv_t * 256 + 128 * h, pv_kvh, pv_b);
+          for (int h = 0; h < 2; ++h)
+            load(&tmV, 4 * m + 2 * (int)cr, pv_t * 256 + 128 * h, pv_kvh, pv_b, pol_v);
       };
       while (ok && w.next(b, kvh, t0, n)) {
         for (int i = 0; i < n && ok; ++i) {
           const int t = t0 + i;
           if (i == 0 && pv_t >= 0) load_v();  // finish the previous piece first
-          for (int c = 0; c < T::KCH; c += 2) load(&tmK, c, t * 256 + 128 * (int)cr, kvh, b);
+          for (int c = 0; c < T::KCH; c += 2) load(&tmK, c, t * 256 + 128 * (int)cr, kvh, b, pol_k);
           if (i > 0) load_v();
           pv_t = t;
           pv_kvh = kvh;
