@@ -206,6 +206,30 @@ void set_smem(K kernel, int bytes) {
 
 enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
 
+// The combine is launched with programmatic stream serialization: its blocks
+// may be scheduled while the split kernel finishes and wait (griddepcontrol)
+// only before reading the partials, so its launch and prologue overlap the
+// split kernel's tail.
+template <bool BF16>
+attn_status_t launch_combine(const attn::DecodeParams& dp, const attn::CombineParams& cp,
+                             cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(dp.B * dp.Hq * dp.Sq), 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16>, cp) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ECUDA;
+  }
+  return ATTN_OK;
+}
+
 template <int DK, int DV, int NH, bool BF16>
 attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
@@ -218,10 +242,7 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
     kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
-  if (phases & PHASE_COMBINE) {
-    attn::combine_kernel<BF16><<<dp.B * dp.Hq * dp.Sq, 128, 0, st>>>(cp);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-  }
+  if (phases & PHASE_COMBINE) return launch_combine<BF16>(dp, cp, st);
   return ATTN_OK;
 }
 
@@ -250,10 +271,7 @@ attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, cons
       return ATTN_ECUDA;
     }
   }
-  if (phases & PHASE_COMBINE) {
-    attn::combine_kernel<BF16><<<dp.B * dp.Hq * dp.Sq, 128, 0, st>>>(cp);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
-  }
+  if (phases & PHASE_COMBINE) return launch_combine<BF16>(dp, cp, st);
   return ATTN_OK;
 }
 

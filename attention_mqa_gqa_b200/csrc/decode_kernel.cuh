@@ -296,6 +296,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the combine may be scheduled now
   locate_range(p.skv, p.B, p.Hkv, 7, p.ranges, rng, scan, sched);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
@@ -752,6 +753,9 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   tot = (redl[4] + redl[5]) + (redl[6] + redl[7]);
   const int tu = key_tiles(p.skv[b], p.tile_shift);
   const long long T = tot * p.Hkv;
+  // Everything above reads inputs only; the partials come from the kernel
+  // before this one in the stream, which may still be running.
+  pdl_wait();
   const long long Re = T < p.ranges ? T : p.ranges;  // ranges in use, none empty
   const long long u = (long long)b * p.Hkv + kvh;
   int n = 0;

@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
     tmem_alloc_pair(smem_u32(tmem_slot), 512);
     tmem_relinquish_pair();
   }
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the combine may be scheduled now
   locate_range(p.skv, p.B, p.Hkv, T::TILE_SHIFT, p.ranges, rng, scan, sched);
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers and the pair's TMEM exist

@@ -145,6 +145,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
   }
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream is still
+// running; pdl_wait() blocks until that kernel has completed and its memory
+// operations are visible.  pdl_launch_dependents() lets the next kernel
+// (if it was launched that way) start early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

@@ -39,9 +39,15 @@ sys.path.insert(0, ROOT)
 
 from attention_mqa_gqa_b200 import workloads as wl  # noqa: E402
 
-KERNEL_SOURCES = ["attention_mqa_gqa_b200/csrc/sm100.cuh", "attention_mqa_gqa_b200/csrc/decode_kernel.cuh",
-                  "attention_mqa_gqa_b200/csrc/mla_pair_kernel.cuh",
-                  "attention_mqa_gqa_b200/csrc/prefill_kernel.cuh", "attention_mqa_gqa_b200/csrc/attn_api.cu"]
+_CSRC = "attention_mqa_gqa_b200/csrc/"
+# the sources each kernel is built from (a committed ncu traffic figure is
+# used only while these are unchanged)
+KERNEL_SOURCES = {
+    "decode_split_kernel": [_CSRC + "sm100.cuh", _CSRC + "decode_kernel.cuh", _CSRC + "attn_api.cu"],
+    "mla_pair_kernel": [_CSRC + "sm100.cuh", _CSRC + "decode_kernel.cuh", _CSRC + "mla_pair_kernel.cuh",
+                        _CSRC + "attn_api.cu"],
+    "prefill_kernel": [_CSRC + "sm100.cuh", _CSRC + "prefill_kernel.cuh", _CSRC + "attn_api.cu"],
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -86,9 +92,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def sources_hash() -> str:
+def sources_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for s in KERNEL_SOURCES:
+    for s in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, s), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -103,7 +109,7 @@ def traffic_for(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel}:{workload}")
-    if not e or e.get("sources_sha") != sources_hash():
+    if not e or e.get("sources_sha") != sources_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
