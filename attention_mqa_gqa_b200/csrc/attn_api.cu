@@ -410,6 +410,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.n_qtiles = (Sq + 127) / 128;
   pp.dv_parts = pl.dv_parts;
   pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;
+  {
+    // K/V bytes of one kv head over the batch; blocks of kv heads whose
+    // K/V stays within ~40 MB of the 126 MB L2
+    const double kv_head_bytes = (double)B * max_skv * (d_k + d_v) * 2.0;
+    int kv_heads = (int)(40.0e6 / (kv_head_bytes > 1.0 ? kv_head_bytes : 1.0));
+    if (kv_heads < 1) kv_heads = 1;
+    if (kv_heads > Hkv) kv_heads = Hkv;
+    pp.heads_per_block = kv_heads * G;
+  }
   pp.scale_log2 = scale_log2;
   pp.causal = causal;
   pp.timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);

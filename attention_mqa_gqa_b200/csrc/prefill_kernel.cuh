@@ -48,6 +48,7 @@ struct PrefillParams {
   const int32_t* skv;         // [B] (device)
   int B, Hq, Hkv, G, Sq;
   int n_qtiles, dv_parts, n_items;
+  int heads_per_block;        // q heads (a multiple of G) whose items run together
   float scale_log2;           // scale * log2(e), scale > 0
   int causal;
   uint64_t timeout_ns;
@@ -57,14 +58,23 @@ struct PrefillItem {
   int part, h, b, kvh, q0, skv, ntiles;
 };
 
-// Work item L (0 = heaviest): the dv parts and heads of one q tile are
-// adjacent so that CTAs running at the same time read the same K/V tiles.
+// Work item L.  The q heads are taken in blocks of heads_per_block whose
+// K/V together fit comfortably in L2 (the items of one block run at about
+// the same time, so each K/V tile comes from DRAM about once); inside a
+// block the heaviest q tiles come first, and the dv parts and heads of one
+// q tile are adjacent so that CTAs running at the same time read the same
+// K/V tiles.
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int L) {
   PrefillItem it;
+  const int per_head = p.n_qtiles * p.B * p.dv_parts;
+  const int blk = L / (p.heads_per_block * per_head);
+  L -= blk * p.heads_per_block * per_head;
+  const int h0 = blk * p.heads_per_block;
+  const int nh = min(p.heads_per_block, p.Hq - h0);  // heads of this block
   it.part = L % p.dv_parts;
   L /= p.dv_parts;
-  it.h = L % p.Hq;
-  L /= p.Hq;
+  it.h = h0 + L % nh;
+  L /= nh;
   it.b = L % p.B;
   const int qt = p.n_qtiles - 1 - L / p.B;
   it.kvh = it.h / p.G;
