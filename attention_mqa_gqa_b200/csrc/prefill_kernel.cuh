@@ -29,12 +29,13 @@
 // mask) with a stride of the grid size, so the next item's Q load and K/V
 // stream overlap the current item's last MMAs and epilogue.
 //
-// Warp roles (320 threads): warp 0 lane 0 streams K/V chunks through a ring
-// of 32 KB groups and lane 1 loads Q per item (TMA), warp 1 allocates TMEM
-// and issues UMMA, warps 2-9 run the softmax, rescale and epilogue: two
-// threads per q row (warps w and w+4 share a TMEM lane quarter), each owning
-// half of the row's keys and half of its output columns, exchanging the row
-// maximum and sum through shared memory.
+// Warp roles: warp 0 lane 0 streams K/V chunks through a ring of 32 KB
+// groups and lane 1 loads Q per item (TMA), warp 1 allocates TMEM and issues
+// UMMA, the other warps (8 at d_k = 512, else 16) run the softmax, rescale
+// and epilogue: SPLIT threads per q row (warps with the same index mod 4
+// share a TMEM lane quarter), each owning a slice of the row's keys and of
+// its output columns, exchanging the row maximum and sum through shared
+// memory.
 #pragma once
 
 #include "sm100.cuh"
@@ -95,8 +96,12 @@ struct PrefillTraits {
   static constexpr int QCH = (KCH + 1) & ~1;     // chunk slots per Q row: pairs, the
                                                  // last one zero-filled if KCH is odd
   static constexpr int VCH = DVH / 64;           // V chunks per key tile (this item's columns)
-  static constexpr int NQ = (DK >= 512) ? 1 : 2;  // Q buffers
-  static constexpr int RING = (DK >= 512 || QCH > 2) ? 6 : 10;  // 16 KB chunk slots
+  // softmax threads per q row: 2 at d_k = 512 (bound by copies and MMA),
+  // 4 otherwise (bound by the softmax's instruction issue: more warps hide
+  // more latency)
+  static constexpr int SPLIT = (DK >= 512) ? 2 : 4;
+  static constexpr int NQ = (DK >= 512 || QCH > 2) ? 1 : 2;  // Q buffers
+  static constexpr int RING = (DK >= 512) ? 6 : 8;            // 16 KB chunk slots
   static constexpr int SLOT = 16384;
   // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
   // copies of a single 16 KB chunk cap a CTA's stream well below what the
@@ -107,13 +112,17 @@ struct PrefillTraits {
   static constexpr int Q_BYTES = QCH * SLOT;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
-  static constexpr int OFF_XCH = OFF_RING + RING * SLOT;     // float [2][128]: row-half exchange
-  static constexpr int OFF_FLAGS = OFF_XCH + 2 * 128 * 4;     // abort, tmem base
+  // row exchange buffers float [XR][SPLIT][128]: two rounds alternate with
+  // the tile (one barrier per exchange); at d_k = 512 shared memory has room
+  // for one round only, which then takes a second barrier
+  static constexpr int XR = (DK >= 512) ? 1 : 2;
+  static constexpr int OFF_XCH = OFF_RING + RING * SLOT;
+  static constexpr int OFF_FLAGS = OFF_XCH + XR * SPLIT * 128 * 4;  // abort, tmem base
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
   // full[RING_G], empty[RING_G], q_full[NQ], q_free[NQ], s_full[2], p_full[2],
   // o_done[2] (one of each per S/P buffer), o_free, drain
   static constexpr int NBAR = 2 * RING_G + 2 * NQ + 8;
-  static constexpr int SOFTMAX_THREADS = 256;    // two threads per q row (64 keys each)
+  static constexpr int SOFTMAX_THREADS = 128 * SPLIT;
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int TMEM_S = 0;               // two S buffers, 128 columns each; P(j)
@@ -127,7 +136,7 @@ struct PrefillTraits {
 };
 
 template <int DK, int DVH, bool BF16>
-__global__ void __launch_bounds__(64 + 256, 1)
+__global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using T = PrefillTraits<DK, DVH>;
@@ -334,18 +343,22 @@ __global__ void __launch_bounds__(64 + 256, 1)
     if (ok && j > 0) pv(j - 1, prev_first, prev_k);
   } else if (warp >= 2) {
     // ---------------------------------------------------- softmax + epilogue
+    // SPLIT threads per q row: warps w with the same w % 4 share a TMEM lane
+    // quarter; quarter-mate qd owns keys [KS qd, KS qd + KS) of each tile and
+    // output columns [HC qd, HC qd + HC).
+    constexpr int SPLIT = T::SPLIT;
+    constexpr int KS = T::KT / SPLIT;        // keys per thread per tile
+    constexpr int HC = DVH / SPLIT;          // output columns per thread
     const int wq = warp & 3;
-    const int half = (warp - 2) >> 2;        // which 64 keys / DVH/2 columns of the row
+    const int qd = (warp - 2) >> 2;          // which slice of the row
     const int row = wq * 32 + lane;          // q row within the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    constexpr int HC = DVH / 2;              // output columns per thread
-    // The two threads of a row meet on named barrier 1 + wq (warps w, w + 4).
-    // A pair barrier waits without bound, so both threads must always reach
-    // the same ones: a failed wait only clears `ok` (skipping the work that
-    // depends on it), and the pair leaves its loops together right after the
-    // next pair barrier that ANDs `ok` over both (pair_and).
-    auto pair_sync = [&]() { named_bar_sync(1 + wq, 64); };
-    auto pair_and = [&](bool v) { return named_bar_and(1 + wq, 64, v); };
+    // The SPLIT threads of a row meet on named barrier 1 + wq.  Such a
+    // barrier waits without bound, so all of them must always reach the
+    // same ones: a failed wait only clears `ok` (skipping the work that
+    // depends on it), and the group leaves its loops together right after
+    // the next barrier that ANDs `ok` over the group (group_and).
+    auto group_and = [&](bool v) { return named_bar_and(1 + wq, 32 * SPLIT, v); };
     volatile int own_abort = 0;
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
       return mbar_wait_warp(bar, parity, &own_abort, p.timeout_ns, id);
@@ -357,52 +370,46 @@ __global__ void __launch_bounds__(64 + 256, 1)
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
       lim = max(0, min(it.skv, lim));
-      float m_used = -INFINITY;  // log2-domain running max (lazily raised), same in both halves
-      float l = 0.f;             // this half's share of the row sum
+      float m_used = -INFINITY;  // log2-domain running max (lazily raised), same in the group
+      float l = 0.f;             // this thread's share of the row sum
 
       for (int i = 0; i < it.ntiles; ++i, ++j) {
         const int sb = j & 1;
         if (ok) ok = wait(s_full + 8 * sb, (j >> 1) & 1, 30);
-        float s[64];
+        float s[KS];
         float mx = -INFINITY;
         if (ok) {
           tc_fence_after();
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float tmp[16];
-            tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + half * 64 + g * 16, tmp);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) s[g * 16 + e] = tmp[e];
-          }
+          tmem_ld<KS>(tmem + lane_base + T::TMEM_S + sb * 128 + qd * KS, s);
           tmem_wait_ld();
 
-          const int kb = i * T::KT + half * 64;
+          const int kb = i * T::KT + qd * KS;
           // Keys at or past `lim` are invisible to this row; only tiles that
           // straddle `lim` need the mask.  The maximum is taken on the raw
           // scores (scale > 0) in 8 independent chains, then scaled once.
-          if (kb + 64 > lim) {
+          if (kb + KS > lim) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
+            for (int c = 0; c < KS; ++c)
               if (kb + c >= lim) s[c] = -INFINITY;
           }
           float mc[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) mc[e] = s[e];
 #pragma unroll
-          for (int c = 8; c < 64; ++c) mc[c & 7] = fmaxf(mc[c & 7], s[c]);
+          for (int c = 8; c < KS; ++c) mc[c & 7] = fmaxf(mc[c & 7], s[c]);
           mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
                      fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
         }
-        // row maximum = max of the two halves (exchanged through smem; the
-        // buffer alternates with the tile so one barrier per tile suffices)
-        float* xb = xch + (j & 1) * 128;
-        if (half == 1) xb[row] = mx;
-        ok = pair_and(ok);
+        // row maximum over the group's slices, exchanged through shared
+        // memory; the buffer alternates with the tile, so the one barrier
+        // per tile also orders the reuse
+        float* xb = xch + (j % T::XR) * (SPLIT * 128);
+        xb[qd * 128 + row] = mx;
+        ok = group_and(ok);
         if (!ok) break;
-        if (half == 0) mx = fmaxf(mx, xb[row]);
-        if (half == 0) xb[row] = mx;
-        pair_sync();
-        if (half == 1) mx = xb[row];
+#pragma unroll
+        for (int k = 0; k < SPLIT; ++k) mx = fmaxf(mx, xb[k * 128 + row]);
+        if (T::XR == 1) named_bar_sync(1 + wq, 32 * SPLIT);  // all have read the round
         mx *= p.scale_log2;
         // Raise the running max only when the tile's exceeds it by more than 8
         // (log2 units); weights stay <= 256 and O/l is unaffected.
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
         const float m_new = need ? mx : m_used;
         const float alpha = need ? ex2(m_used - m_new) : 1.f;
         const bool warp_need = __any_sync(0xffffffffu, need);
-        // a failed wait ends the tile here and the pair leaves at the next pair_and
+        // a failed wait ends the tile here and the group leaves at the next group_and
         if (warp_need && i > 0) {  // rescale this thread's O columns once PV(j-1) landed
           const int t = j - 1;
           ok = wait(o_done + 8 * (t & 1), (t >> 1) & 1, 32);
@@ -419,7 +426,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
 #pragma unroll 1
           for (int g = 0; g < HC / 16; ++g) {
             float o[16];
-            const uint32_t ta = tmem + lane_base + T::TMEM_O + half * HC + g * 16;
+            const uint32_t ta = tmem + lane_base + T::TMEM_O + qd * HC + g * 16;
             tmem_ld16(ta, o);
             tmem_wait_ld();
 #pragma unroll
@@ -431,9 +438,9 @@ __global__ void __launch_bounds__(64 + 256, 1)
         l *= alpha;
         m_used = m_new;
 
-        // P row half -> TMEM columns [32 * half, 32 * half + 32) of S buffer sb
-        // (two bf16 per column, keys in order; both halves of the row have read
-        // their S values before the pair barrier above):
+        // P slice -> TMEM columns [KS/2 qd, KS/2 qd + KS/2) of S buffer sb (two
+        // bf16 per column, keys in order; the whole group has read its S
+        // values before the barrier above):
         // p = exp2(s * scale * log2e - m), one FMA and one SFU op per key; a row
         // that has seen no visible key yet (m = -inf) writes zeros.
         const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
@@ -442,7 +449,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) lc[e] = 0.f;
 #pragma unroll
-        for (int h16 = 0; h16 < 2; ++h16) {
+        for (int h16 = 0; h16 < KS / 32; ++h16) {
           float u[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -453,7 +460,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
             lc[(2 * e) & 7] += p0;
             lc[(2 * e + 1) & 7] += p1;
           }
-          tmem_st16(tmem + lane_base + T::TMEM_S + sb * 128 + half * 32 + h16 * 16, u);
+          tmem_st16(tmem + lane_base + T::TMEM_S + sb * 128 + qd * (KS / 2) + h16 * 16, u);
         }
         l += ((lc[0] + lc[1]) + (lc[2] + lc[3])) + ((lc[4] + lc[5]) + (lc[6] + lc[7]));
         tmem_wait_st();
@@ -462,31 +469,31 @@ __global__ void __launch_bounds__(64 + 256, 1)
       }
 
       // ------------------------------------------------------ epilogue
-      // row sum = both halves (the exchange buffer of this round is free:
-      // its last readers passed the second pair barrier of the last tile)
-      float* xb = xch + (j & 1) * 128;
-      if (half == 1) xb[row] = l;
-      ok = pair_and(ok);
+      // row sum over the group (this round's exchange buffer is free: its
+      // last readers passed the barrier of the last tile)
+      float* xb = xch + (j % T::XR) * (SPLIT * 128);
+      xb[qd * 128 + row] = l;
+      ok = group_and(ok);
       if (!ok) break;
-      const float lrow = half == 0 ? l + xb[row] : 0.f;
-      if (half == 0) xb[row] = lrow;
-      pair_sync();
-      const float ltot = half == 0 ? lrow : xb[row];
+      float ltot = 0.f;
+#pragma unroll
+      for (int k = 0; k < SPLIT; ++k) ltot += xb[k * 128 + row];
+      if (T::XR == 1) named_bar_sync(1 + wq, 32 * SPLIT);
       if (it.ntiles > 0) {
         const int t = j - 1;
         ok = wait(o_done + 8 * (t & 1), (t >> 1) & 1, 33);
-        if (!ok) continue;  // no pair barrier before the next item's first pair_and
+        if (!ok) continue;  // no group barrier before the next item's first group_and
         tc_fence_after();
       }
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
                       ((int64_t)it.b * p.o_sb + (int64_t)it.h * p.o_sh + (int64_t)qi * p.o_ss +
-                       it.part * DVH + half * HC) * 2;
+                       it.part * DVH + qd * HC) * 2;
 #pragma unroll 1
       for (int g = 0; g < HC / 16; ++g) {
         float o[16];
         if (it.ntiles > 0) {
-          tmem_ld16(tmem + lane_base + T::TMEM_O + half * HC + g * 16, o);
+          tmem_ld16(tmem + lane_base + T::TMEM_O + qd * HC + g * 16, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -505,7 +512,7 @@ __global__ void __launch_bounds__(64 + 256, 1)
         tc_fence_before();
         mbar_arrive(o_free);
       }
-      if (half == 0 && it.part == 0 && p.lse && qi < p.Sq)
+      if (qd == 0 && it.part == 0 && p.lse && qi < p.Sq)
         p.lse[((int64_t)it.b * p.Hq + it.h) * p.Sq + qi] =
             ltot > 0.f ? (m_used + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
     }
