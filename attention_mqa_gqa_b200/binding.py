@@ -15,7 +15,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
 
-ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_EWORKSPACE, ATTN_ECUDA, ATTN_ETIMEOUT = range(6)
+(ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_EWORKSPACE, ATTN_ECUDA, ATTN_ETIMEOUT,
+ ATTN_EOVERFLOW) = range(7)
 ATTN_BF16, ATTN_FP16 = 0, 1
 
 
@@ -42,7 +43,7 @@ class AttnError(RuntimeError):
 # Every symbol include/attn_b200.h declares (checked by the CPU test suite).
 EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
            "attn_decode_combine", "attn_fwd_noalloc", "attn_last_device_error", "attn_status_str",
-           "attn_version", "attn_set_wait_timeout_ns")
+           "attn_version", "attn_set_wait_timeout_ns", "attn_cache_append")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in the header
 
 _lib = None
@@ -71,6 +72,9 @@ def load(path: str | None = None):
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, i32, i32,
                                      ctypes.c_float, i32, i32, Strides, Strides, Strides,
                                      Strides, vp]
+    lib.attn_cache_append.restype = i32
+    lib.attn_cache_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, Strides,
+                                      Strides, Strides, Strides, vp]
     lib.attn_set_wait_timeout_ns.restype = ctypes.c_uint64
     lib.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.attn_last_device_error.restype = i32
@@ -183,6 +187,30 @@ def attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: tor
 def last_device_error(stream: torch.cuda.Stream | None = None) -> int:
     st = stream if stream is not None else torch.cuda.current_stream()
     return int(load().attn_last_device_error(st.cuda_stream))
+
+
+def cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor | None, k_new: torch.Tensor,
+                 v_new: torch.Tensor | None, skv: torch.Tensor,
+                 stream: torch.cuda.Stream | None = None) -> None:
+    """attn_cache_append: write k_new[b, h] (and v_new[b, h]) at position
+    skv[b] of the caches and advance skv (device-side).  k_cache/v_cache are
+    [B, Hkv, max_skv, d] (views allowed); for an MLA latent cache pass the
+    same tensor (or None) as v_cache.  k_new/v_new are [B, Hkv, 1, d]."""
+    B, Hkv, max_skv, d_k = k_cache.shape
+    if skv.dtype != torch.int32:
+        raise TypeError("skv must be int32")
+    latent = v_cache is None or v_cache.data_ptr() == k_cache.data_ptr()
+    d_v = 0 if latent else v_cache.shape[-1]
+    st = stream if stream is not None else torch.cuda.current_stream(k_cache.device)
+    zero = Strides(0, 0, 0)
+    rc = load().attn_cache_append(k_cache.data_ptr(), None if latent else v_cache.data_ptr(),
+                                  k_new.data_ptr(), None if latent else v_new.data_ptr(),
+                                  skv.data_ptr(), B, Hkv, max_skv, d_k, d_v,
+                                  dtype_code(k_cache.dtype), _strides4(k_cache),
+                                  zero if latent else _strides4(v_cache), _strides4(k_new),
+                                  zero if latent else _strides4(v_new), st.cuda_stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_cache_append")
 
 
 def set_wait_timeout_ns(ns: int) -> int:

@@ -15,6 +15,7 @@
 
 #include "../../include/attn_b200.h"
 #include "decode_kernel.cuh"
+#include "cache_append.cuh"
 #include "mla_pair_kernel.cuh"
 #include "prefill_kernel.cuh"
 
@@ -475,7 +476,8 @@ attn_status_t attn_last_device_error(void* cuda_stream) {
     return ATTN_ECUDA;
   if (word != 0 && cudaMemcpyToSymbol(attn::g_attn_error, &zero, sizeof(zero)) != cudaSuccess)
     return ATTN_ECUDA;
-  return word ? ATTN_ETIMEOUT : ATTN_OK;
+  if (word & 1u) return ATTN_ETIMEOUT;
+  return word ? ATTN_EOVERFLOW : ATTN_OK;
 }
 
 const char* attn_status_str(attn_status_t s) {
@@ -486,11 +488,55 @@ const char* attn_status_str(attn_status_t s) {
     case ATTN_EWORKSPACE: return "workspace missing or too small";
     case ATTN_ECUDA: return "CUDA error";
     case ATTN_ETIMEOUT: return "device-side wait timed out";
+    case ATTN_EOVERFLOW: return "cache full: a sequence already holds max_skv keys";
   }
   return "unknown status";
 }
 
 const char* attn_version(void) { return "0.1.0"; }
+
+attn_status_t attn_cache_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                                int32_t* skv_per_seq, int B, int Hkv, int max_skv, int d_k,
+                                int d_v, attn_dtype_t dtype, attn_strides_t sk, attn_strides_t sv,
+                                attn_strides_t skn, attn_strides_t svn, void* cuda_stream) {
+  if (!k_cache || !k_new || !skv_per_seq) return ATTN_EINVAL;
+  if (B <= 0 || Hkv <= 0 || max_skv <= 0 || d_k <= 0 || d_v < 0) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_EINVAL;
+  if (d_k % 8 != 0 || d_v % 8 != 0) return ATTN_EINVAL;
+  if (reinterpret_cast<uintptr_t>(skv_per_seq) & 3u) return ATTN_EINVAL;
+  // v_cache == NULL or == k_cache with d_v <= d_k: the MLA latent cache,
+  // where V is a view of K's rows -- only the K row is written
+  const bool write_v = v_cache && v_cache != k_cache && d_v > 0;
+  if (write_v && !v_new) return ATTN_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(k_new) || (write_v && (!aligned16(v_cache) || !aligned16(v_new))))
+    return ATTN_EINVAL;
+  if (!strides_ok(sk) || !strides_ok(skn) || (write_v && (!strides_ok(sv) || !strides_ok(svn))))
+    return ATTN_EINVAL;
+  attn::AppendParams ap{};
+  ap.kc = reinterpret_cast<uint8_t*>(k_cache);
+  ap.vc = reinterpret_cast<uint8_t*>(v_cache);
+  ap.kn = reinterpret_cast<const uint8_t*>(k_new);
+  ap.vn = reinterpret_cast<const uint8_t*>(v_new);
+  ap.skv = skv_per_seq;
+  ap.B = B;
+  ap.Hkv = Hkv;
+  ap.max_skv = max_skv;
+  ap.dk = d_k;
+  ap.dv = d_v;
+  ap.write_v = write_v ? 1 : 0;
+  ap.k_sb = sk.b;
+  ap.k_sh = sk.h;
+  ap.k_ss = sk.s;
+  ap.v_sb = sv.b;
+  ap.v_sh = sv.h;
+  ap.v_ss = sv.s;
+  ap.kn_sb = skn.b;
+  ap.kn_sh = skn.h;
+  ap.vn_sb = svn.b;
+  ap.vn_sh = svn.h;
+  attn::cache_append_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(ap);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
 
 uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
   return g_wait_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);

@@ -62,7 +62,8 @@ typedef enum {
   ATTN_EUNSUPPORTED = 2,  /* valid request outside the supported shapes        */
   ATTN_EWORKSPACE = 3,    /* workspace missing or smaller than required        */
   ATTN_ECUDA = 4,         /* a CUDA runtime/driver call or launch failed       */
-  ATTN_ETIMEOUT = 5       /* a device-side wait gave up (see attn_last_device_error) */
+  ATTN_ETIMEOUT = 5,      /* a device-side wait gave up (see attn_last_device_error) */
+  ATTN_EOVERFLOW = 6      /* attn_cache_append found a full sequence (see attn_last_device_error) */
 } attn_status_t;
 
 typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype_t;
@@ -186,10 +187,36 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void
  * Synchronises `cuda_stream`, then reads and clears the current device's
  * error word.  ATTN_OK if no kernel of this library reported a problem
  * since the last call, ATTN_ETIMEOUT if a device-side wait gave up (the
- * outputs of that launch are undefined), ATTN_ECUDA if the stream itself
- * reports an error.
+ * outputs of that launch are undefined), ATTN_EOVERFLOW if attn_cache_append
+ * met a full sequence, ATTN_ECUDA if the stream itself reports an error.
  */
 attn_status_t attn_last_device_error(void* cuda_stream);
+
+/*
+ * Append the new token's cached row(s) before a decode step ("Full 路线"
+ * section 三: past_key_value.update, then attention over the whole cache;
+ * sections 4.2-4.3: in MLA the cached row is [c_kv | k_pe]).  For every
+ * sequence b whose length skv[b] < max_skv, and every kv head h, copies
+ * k_new[b, h, :] (d_k elements) to k_cache[b, h, skv[b], :] and
+ * v_new[b, h, :] (d_v elements) to v_cache[b, h, skv[b], :], then sets
+ * skv[b] += 1 -- all on `cuda_stream`, so an attn_fwd enqueued after it on
+ * the same stream attends over the new key as well.
+ * - k_cache/v_cache: [B, Hkv, max_skv, d] with element strides sk / sv
+ *   (innermost contiguous); k_new/v_new: [B, Hkv, 1, d] with strides skn /
+ *   svn (the s stride is ignored).  skv_per_seq: device int32 [B], updated.
+ * - MLA latent cache: pass v_cache == k_cache (or NULL); only the K row (the
+ *   whole [c_kv | k_pe] row, d_k = 576) is written and v_new is ignored.
+ * - A sequence already holding max_skv keys is left unchanged and bit 1 of
+ *   the device error word is set: attn_last_device_error then returns
+ *   ATTN_EOVERFLOW.
+ * - Errors before launch: ATTN_EINVAL (null or misaligned pointers, strides
+ *   or d not multiples of 8 elements, bad dtype); ATTN_ECUDA on a launch error.
+ * The pages have no counterpart beyond the cache update they call.
+ */
+attn_status_t attn_cache_append(void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                                int32_t* skv_per_seq, int B, int Hkv, int max_skv, int d_k,
+                                int d_v, attn_dtype_t dtype, attn_strides_t sk, attn_strides_t sv,
+                                attn_strides_t skn, attn_strides_t svn, void* cuda_stream);
 
 /* Bound on every device-side wait of launches made after this call, in
  * nanoseconds of %globaltimer (process-wide; 0 restores the default of 2 s).

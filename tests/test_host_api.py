@@ -33,7 +33,7 @@ def test_header_declarations_are_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert binding.status_str(code) and binding.status_str(code) != "unknown status"
     assert binding.version().count(".") == 2
 
@@ -189,3 +189,25 @@ def _call(lib, **over):
 ])
 def test_fwd_rejects_before_launch(lib, over, code):
     assert _call(lib, **over) == code
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(kc=None), binding.ATTN_EINVAL),
+    (dict(skv=None), binding.ATTN_EINVAL),
+    (dict(dk=100), binding.ATTN_EINVAL),                 # not a multiple of 8 elements
+    (dict(kn=0x20008), binding.ATTN_EINVAL),             # not 16-byte aligned
+    (dict(vn=None), binding.ATTN_EINVAL),                # separate V cache needs v_new
+    (dict(B=0), binding.ATTN_EINVAL),
+    (dict(dtype=9), binding.ATTN_EINVAL),
+])
+def test_cache_append_rejects_before_launch(lib, over, code):
+    """attn_cache_append validates its arguments before anything reaches the
+    device (the fake pointers below are never dereferenced)."""
+    a = dict(kc=0x10000, vc=0x30000, kn=0x20000, vn=0x40000, skv=0x50000, B=2, Hkv=1,
+             max_skv=64, dk=128, dv=128, dtype=0)
+    a.update(over)
+    s = binding.Strides(64 * 128, 64 * 128, 128)
+    sn = binding.Strides(128, 128, 128)
+    assert lib.attn_cache_append(a["kc"], a["vc"], a["kn"], a["vn"], a["skv"], a["B"], a["Hkv"],
+                                 a["max_skv"], a["dk"], a["dv"], a["dtype"], s, s, sn, sn,
+                                 None) == code
