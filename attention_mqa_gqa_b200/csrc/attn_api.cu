@@ -128,9 +128,9 @@ bool strides_ok(const attn_strides_t& s) {
 }
 
 // Resident decode CTAs per SM (must match DecodeTraits<...>::CTAS).
-// Decode CTAs resident per SM: two for d_k in {128, 512}; for MLA (576) one
-// CTA per SM, the SMs working in pairs (each pair one cluster of two CTAs).
-int decode_ctas_per_sm(int d_k) { return d_k == 576 ? 1 : 2; }
+// Decode CTAs resident per SM: two for d_k = 128, one for 512; for MLA (576)
+// one CTA per SM, the SMs working in pairs (each pair one cluster of two CTAs).
+int decode_ctas_per_sm(int d_k) { return d_k == 128 ? 2 : 1; }
 bool decode_pairs(int d_k) { return d_k == 576; }
 
 bool shape_supported(int Sq, int d_k, int d_v) {
@@ -236,7 +236,7 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
                             const attn_plan_t& pl, cudaStream_t st, int phases) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
-  static_assert(Tr::CTAS == 2 && DK != 576, "decode_ctas_per_sm out of sync");
+  static_assert(Tr::CTAS == (DK == 128 ? 2 : 1) && DK != 576, "decode_ctas_per_sm out of sync");
   if (phases & PHASE_PARTIAL) {
     auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
     set_smem(kern, Tr::SMEM_BYTES);

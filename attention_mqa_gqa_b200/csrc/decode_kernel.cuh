@@ -76,8 +76,11 @@ struct DecodeTraits {
   static constexpr int KG = (KCH + GCH - 1) / GCH;  // ring groups per K tile
   static constexpr int VG = VCH / GCH;              // ring groups per V tile (one per O^T block)
   static constexpr int DVB = DV / 128;             // 128-row blocks of O^T
-  static constexpr int CTAS = (DK == 576) ? 1 : 2; // resident CTAs per SM
-  static constexpr int RING = (DK == 576) ? 6 : (DK == 512 ? 4 : 6);
+  // resident CTAs per SM: at d = 512 one CTA per SM with a deeper ring
+  // (with ~8 key tiles per range instead of ~4 the tiles split more evenly
+  // over the ranges); at d = 128 two
+  static constexpr int CTAS = (DK == 128) ? 2 : 1;
+  static constexpr int RING = (DK == 512) ? 8 : 6;
   static constexpr int NPT = 2;                    // P^T buffers
   static constexpr int SOFTMAX_THREADS = 256;      // two threads per key row
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;

@@ -50,7 +50,7 @@ def test_plan_decode_invariants(lib):
         assert pl["heads_per_cta"] == (128 if dk == 576 else 16)
         assert pl["head_blocks"] == -(-G // pl["heads_per_cta"])
         ctas_per_range = 2 if dk == 576 else 1
-        ctas_per_sm = 1 if dk == 576 else 2
+        ctas_per_sm = 2 if dk == 128 else 1
         assert pl["kv_ranges"] == max(1, 148 * ctas_per_sm // ctas_per_range // pl["head_blocks"])
         assert pl["grid_ctas"] == pl["kv_ranges"] * pl["head_blocks"] * ctas_per_range
         assert pl["partials"] == pl["kv_ranges"] + B * Hkv
