@@ -54,7 +54,8 @@ EncodeTiledFn get_encode_fn() {
 // limited per CTA well below HBM bandwidth).  D must be a multiple of 64;
 // chunks past D/64 are out of range and zero-filled.
 bool make_chunk_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_t D, uint64_t S,
-                    uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb, uint32_t kch) {
+                    uint64_t H, uint64_t B, int64_t ss, int64_t sh, int64_t sb, uint32_t kch,
+                    uint32_t rows = 128) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc || D % 64 != 0) return false;
   if (S == 1) ss = (int64_t)D;
@@ -62,7 +63,7 @@ bool make_chunk_map(CUtensorMap* map, const void* base, attn_dtype_t dt, uint64_
   if (B == 1) sb = sh * (int64_t)H;
   cuuint64_t dims[5] = {64, S, D / 64, H, B};
   cuuint64_t strides[4] = {(cuuint64_t)ss * 2, 128, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
-  cuuint32_t box[5] = {64, 128, kch, 1, 1};
+  cuuint32_t box[5] = {64, rows, kch, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                    5, const_cast<void*>(base), dims, strides, box, estr,
@@ -143,6 +144,11 @@ bool shape_supported(int Sq, int d_k, int d_v) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// d = 512 prefill of groups with an even number of query heads runs on SM
+// pairs (two heads of a kv group per cluster; the K/V copies split between
+// the two SMs).
+bool prefill_pairs(int d_k, int G) { return d_k == 512 && G % 2 == 0; }
+
 // Columns (head x query) per decode CTA for d_k in {128, 512}.
 constexpr int kDecodeCols = 16;
 
@@ -173,7 +179,12 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
     const int64_t n_qt = (Sq + 127) / 128;
     const int64_t items = n_qt * Hq * (int64_t)B * pl->dv_parts;  // persistent CTAs walk these
     if (items > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
-    pl->grid_ctas = items < num_sms ? items : num_sms;
+    if (prefill_pairs(d_k, G)) {  // clusters of two CTAs, one item per pair of heads
+      const int64_t units = items / 2, pairs = num_sms / 2;
+      pl->grid_ctas = 2 * (units < pairs ? units : pairs);
+    } else {
+      pl->grid_ctas = items < num_sms ? items : num_sms;
+    }
     pl->workspace_bytes = 0;
     return ATTN_OK;
   }
@@ -276,13 +287,32 @@ attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, cons
   return ATTN_OK;
 }
 
-template <int DK, int DVH, bool BF16>
+template <int DK, int DVH, bool BF16, bool PAIR = false>
 attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                              const attn::PrefillParams& pp, const attn_plan_t& pl,
                              cudaStream_t st) {
-  using Tr = attn::PrefillTraits<DK, DVH>;
-  auto kern = attn::prefill_kernel<DK, DVH, BF16>;
+  using Tr = attn::PrefillTraits<DK, DVH, PAIR>;
+  auto kern = attn::prefill_kernel<DK, DVH, BF16, PAIR>;
   set_smem(kern, Tr::SMEM_BYTES);
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
+    cfg.blockDim = dim3(Tr::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ECUDA;
+    }
+    return ATTN_OK;
+  }
   kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   return ATTN_OK;
@@ -392,7 +422,11 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
                 : launch_mla_pair<false>(mq, mk, mv, dp, cp, pl, st, phases);
   }
 
-  if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, 2)) return ATTN_ECUDA;
+  const bool pairs = prefill_pairs(d_k, G);
+  // pairs: each CTA copies 64 of a K tile's 128 keys (four chunks per copy)
+  if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, pairs ? 4 : 2,
+                      pairs ? 64 : 128))
+    return ATTN_ECUDA;
   if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
   CUtensorMap mq;
   if (!make_chunk_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b, 2)) return ATTN_ECUDA;
@@ -410,7 +444,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.Sq = Sq;
   pp.n_qtiles = (Sq + 127) / 128;
   pp.dv_parts = pl.dv_parts;
-  pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;
+  pp.pairs = pairs ? 1 : 0;
+  pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts / (pairs ? 2 : 1);  // per CTA or per pair
   {
     // K/V bytes of one kv head over the batch; blocks of kv heads whose
     // K/V stays within ~40 MB of the 126 MB L2
@@ -429,6 +464,9 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   if (d_k == 192)
     return bf16 ? launch_prefill<192, 128, true>(mq, mk, mv, pp, pl, st)
                 : launch_prefill<192, 128, false>(mq, mk, mv, pp, pl, st);
+  if (pairs)
+    return bf16 ? launch_prefill<512, 256, true, true>(mq, mk, mv, pp, pl, st)
+                : launch_prefill<512, 256, false, true>(mq, mk, mv, pp, pl, st);
   return bf16 ? launch_prefill<512, 256, true>(mq, mk, mv, pp, pl, st)
               : launch_prefill<512, 256, false>(mq, mk, mv, pp, pl, st);
 }

@@ -50,6 +50,7 @@ struct PrefillParams {
   int B, Hq, Hkv, G, Sq;
   int n_qtiles, dv_parts, n_items;
   int heads_per_block;        // q heads (a multiple of G) whose items run together
+  int pairs;                  // 1: a cluster of two CTAs takes two heads of one kv group
   float scale_log2;           // scale * log2(e), scale > 0
   int causal;
   uint64_t timeout_ns;
@@ -65,16 +66,20 @@ struct PrefillItem {
 // block the heaviest q tiles come first, and the dv parts and heads of one
 // q tile are adjacent so that CTAs running at the same time read the same
 // K/V tiles.
-__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int L) {
+// With pairs, "heads" below are head pairs (2u, 2u + 1) and CTA `cr` of the
+// pair takes head 2u + cr.
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int L, int cr = 0) {
   PrefillItem it;
+  const int U = p.pairs ? 2 : 1;
+  const int units = p.Hq / U, units_per_block = p.heads_per_block / U;
   const int per_head = p.n_qtiles * p.B * p.dv_parts;
-  const int blk = L / (p.heads_per_block * per_head);
-  L -= blk * p.heads_per_block * per_head;
-  const int h0 = blk * p.heads_per_block;
-  const int nh = min(p.heads_per_block, p.Hq - h0);  // heads of this block
+  const int blk = L / (units_per_block * per_head);
+  L -= blk * units_per_block * per_head;
+  const int h0 = blk * units_per_block;
+  const int nh = min(units_per_block, units - h0);  // head units of this block
   it.part = L % p.dv_parts;
   L /= p.dv_parts;
-  it.h = h0 + L % nh;
+  it.h = (h0 + L % nh) * U + cr;
   L /= nh;
   it.b = L % p.B;
   const int qt = p.n_qtiles - 1 - L / p.B;
@@ -88,7 +93,11 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   return it;
 }
 
-template <int DK, int DVH>
+// PAIR: clusters of two CTAs on two SMs run the MMAs as one (cta_group::2):
+// M = 256 = the two CTAs' q tiles (two heads of one kv group, same rows),
+// and the B operands are split between them -- each CTA copies 64 of a K
+// tile's 128 keys and 128 of V's DVH = 256 columns, half the per-SM copies.
+template <int DK, int DVH, bool PAIR = false>
 struct PrefillTraits {
   static constexpr int TILE = 128;               // q rows per item (MMA M)
   static constexpr int KT = 128;                 // keys per tile (MMA N of S)
@@ -129,17 +138,24 @@ struct PrefillTraits {
                                                  // overwrites the first 64 of S(j)
   static constexpr int TMEM_O = 256;             // DVH columns
   static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int K_ROWS = PAIR ? 64 : 128;      // K rows this CTA copies per tile
+  static constexpr int K_GCH = PAIR ? 4 : GCH;        // K chunks per copy (32 KB)
+  static constexpr int V_CH = PAIR ? 2 : VCH;         // V chunks this CTA copies per tile
+  static_assert(!PAIR || (DK == 512 && DVH == 256), "pairs: d = 512 prefill");
   static_assert(VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
                 "chunks travel in pairs; a V pair is one 128-column block of O");
   static_assert(TMEM_O + DVH <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int DK, int DVH, bool BF16>
-__global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
+template <int DK, int DVH, bool BF16, bool PAIR = false>
+__global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using T = PrefillTraits<DK, DVH>;
+  using T = PrefillTraits<DK, DVH, PAIR>;
+  const uint32_t cr = PAIR ? cluster_ctarank() : 0u;  // PAIR: 0 issues the pair MMAs
+  const int item0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int istride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -175,22 +191,36 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(p_full + 8 * i, T::SOFTMAX_THREADS);
+      mbar_init(p_full + 8 * i, (PAIR ? 2 : 1) * T::SOFTMAX_THREADS);
       mbar_init(o_done + 8 * i, 1);
     }
-    mbar_init(o_free, T::SOFTMAX_THREADS);
+    mbar_init(o_free, (PAIR ? 2 : 1) * T::SOFTMAX_THREADS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), T::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // waits on phases that the other CTA of a pair may complete use cluster scope
+  auto wait1 = [&](uint32_t bar, uint32_t parity, volatile int* ab, uint32_t id) {
+    return PAIR ? mbar_wait_cluster(bar, parity, ab, p.timeout_ns, id)
+                : mbar_wait(bar, parity, ab, p.timeout_ns, id);
+  };
+  auto waitw = [&](uint32_t bar, uint32_t parity, volatile int* ab, uint32_t id) {
+    return PAIR ? mbar_wait_warp_cluster(bar, parity, ab, p.timeout_ns, id)
+                : mbar_wait_warp(bar, parity, ab, p.timeout_ns, id);
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------- producer: K/V ring
@@ -201,29 +231,40 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     uint32_t ph = 0;
     bool ok = true;
     // chunks [ch, ch + GCH) of key rows [row, row + 128) -> the next ring group
+    // one copy (32 KB) starting at chunk `ch` of rows `row`.. -> the next
+    // ring group; with pairs the bytes of both CTAs' copies are counted on
+    // CTA 0's barrier
     auto load = [&](const CUtensorMap* map, int ch, int row, int kvh, int b) {
       if (!ok) return;
-      ok = mbar_wait(empty_bar(grp), ph ^ 1u, abort_flag, p.timeout_ns, 21);
+      ok = wait1(empty_bar(grp), ph ^ 1u, abort_flag, 21);
       if (!ok) return;
-      mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
-      tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, row, ch, kvh, b, pol_kv);
+      if constexpr (PAIR) {
+        if (cr == 0) mbar_arrive_expect_tx(full_bar(grp), 2 * T::GBYTES);
+        tma_load_5d_pair(ring + grp * T::GBYTES, map, mapa_shared(full_bar(grp), 0), 0, row, ch,
+                         kvh, b, pol_kv);
+      } else {
+        mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
+        tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, row, ch, kvh, b, pol_kv);
+      }
       if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
     };
     bool have_prev = false;
     int pv_tok = 0, pv_kvh = 0, pv_b = 0, pv_ch = 0;  // tile whose V is still to load
     auto load_v = [&]() {
-      for (int c = 0; c < T::VCH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
+      for (int c = 0; c < T::V_CH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
     };
-    for (int L = blockIdx.x; L < p.n_items && ok; L += gridDim.x) {
-      const PrefillItem it = prefill_item(p, L);
+    for (int L = item0; L < p.n_items && ok; L += istride) {
+      const PrefillItem it = prefill_item(p, L, (int)cr);
       for (int j = 0; j < it.ntiles && ok; ++j) {
         if (j == 0 && have_prev) load_v();  // finish the previous item first
-        for (int c = 0; c < T::KCH; c += T::GCH) load(&tmK, c, j * T::KT, it.kvh, it.b);
+        for (int c = 0; c < T::KCH; c += T::K_GCH)
+          load(&tmK, c, j * T::KT + (int)cr * T::K_ROWS, it.kvh, it.b);
         if (j > 0) load_v();
         pv_tok = j * T::KT;
         pv_kvh = it.kvh;
         pv_b = it.b;
-        pv_ch = it.part * (DVH / 64);
+        // pairs: this CTA's half of the part's DVH columns
+        pv_ch = it.part * (DVH / 64) + (int)cr * T::V_CH;
         have_prev = true;
       }
     }
@@ -234,24 +275,42 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     const uint64_t pol_q = l2_policy_evict_first();
     int kq = 0;
     bool ok = true;
-    for (int L = blockIdx.x; L < p.n_items && ok; L += gridDim.x) {
-      const PrefillItem it = prefill_item(p, L);
+    for (int L = item0; L < p.n_items && ok; L += istride) {
+      const PrefillItem it = prefill_item(p, L, (int)cr);
       if (it.ntiles == 0) continue;
       const int qb = kq % T::NQ;
       if (kq >= T::NQ)  // buffer qb was last read by the S MMAs of item kq - NQ
-        ok = mbar_wait(q_free + 8 * qb, ((kq - T::NQ) / T::NQ) & 1, abort_flag, p.timeout_ns, 22);
+        ok = wait1(q_free + 8 * qb, ((kq - T::NQ) / T::NQ) & 1, abort_flag, 22);
       if (!ok) break;
-      mbar_arrive_expect_tx(q_full + 8 * qb, T::Q_BYTES);
-      for (int c = 0; c < T::QCH; c += T::GCH)
-        tma_load_5d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, 0, it.q0, c,
-                    it.h, it.b, pol_q);
+      if constexpr (PAIR) {
+        if (cr == 0) mbar_arrive_expect_tx(q_full + 8 * qb, 2 * T::Q_BYTES);
+        const uint32_t lead = mapa_shared(q_full + 8 * qb, 0);
+        for (int c = 0; c < T::QCH; c += T::GCH)
+          tma_load_5d_pair(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, lead, 0, it.q0, c, it.h,
+                           it.b, pol_q);
+      } else {
+        mbar_arrive_expect_tx(q_full + 8 * qb, T::Q_BYTES);
+        for (int c = 0; c < T::QCH; c += T::GCH)
+          tma_load_5d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, 0, it.q0, c,
+                      it.h, it.b, pol_q);
+      }
       ++kq;
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 && (!PAIR || cr == 0)) {
     // ---------------------------------------------------- MMA issuer (whole warp,
     // one elected lane issues; waits are polled by the converged warp)
-    constexpr uint32_t idS = umma_idesc(128, 128, BF16, false, false);  // Q, K both K-major
-    constexpr uint32_t idO = umma_idesc(128, 128, BF16, false, true);   // P K-major, V MN-major
+    constexpr int M = PAIR ? 256 : 128;                                   // pairs: both q tiles
+    constexpr uint32_t idS = umma_idesc(M, 128, BF16, false, false);      // Q, K both K-major
+    constexpr uint32_t idO = umma_idesc(M, PAIR ? 256 : 128, BF16, false, true);  // P K, V MN-major
+    auto mma_ss = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+      if constexpr (PAIR) umma_ss_pair(d, a, b, id, acc); else umma_ss(d, a, b, id, acc);
+    };
+    auto mma_ts = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+      if constexpr (PAIR) umma_ts_pair(d, a, b, id, acc); else umma_ts(d, a, b, id, acc);
+    };
+    auto commit = [&](uint32_t bar) {
+      if constexpr (PAIR) umma_commit_pair(bar); else umma_commit(bar);
+    };
     int grp = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -260,13 +319,13 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     auto pv = [&](int t, bool first, int k) {
       if (!ok) return;
       const int pb = t & 1;
-      ok = mbar_wait_warp(p_full + 8 * pb, (t >> 1) & 1, abort_flag, p.timeout_ns, 23);
-      if (ok && first && k > 0) ok = mbar_wait_warp(o_free, (k - 1) & 1, abort_flag, p.timeout_ns, 24);
+      ok = waitw(p_full + 8 * pb, (t >> 1) & 1, abort_flag, 23);
+      if (ok && first && k > 0) ok = waitw(o_free, (k - 1) & 1, abort_flag, 24);
       if (!ok) return;
       tc_fence_after();
       const uint32_t pcol = tmem + T::TMEM_S + pb * 128;  // P(t): 8 columns per 16 keys
-      for (int i = 0; i < T::VCH / 2; ++i) {
-        ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 25);
+      for (int i = 0; i < T::V_CH / 2; ++i) {  // pairs: one group, N = 256 across the pair
+        ok = waitw(full_bar(grp), ph, abort_flag, 25);
         if (!ok) return;
         tc_fence_after();
         const uint32_t bbase = ring + grp * T::GBYTES;
@@ -276,62 +335,65 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
           // (SBO), 16 keys per K step = 2048 bytes.  A = P(t) from TMEM.
           const uint64_t bd0 = umma_sdesc(bbase, T::SLOT, 1024, SMEM_SW128);
           const uint32_t d = tmem + T::TMEM_O + i * 128;
-          umma_ts(d, pcol, bd0, idO, first ? 0u : 1u);
+          mma_ts(d, pcol, bd0, idO, first ? 0u : 1u);
 #pragma unroll
           for (int ks = 1; ks < 8; ++ks)
-            umma_ts(d, pcol + ks * 8, bd0 + (uint64_t)(ks * (2048 >> 4)), idO, 1u);
-          umma_commit(empty_bar(grp));
+            mma_ts(d, pcol + ks * 8, bd0 + (uint64_t)(ks * (2048 >> 4)), idO, 1u);
+          commit(empty_bar(grp));
         }
         __syncwarp();
         if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
       }
-      if (elect_one()) umma_commit(o_done + 8 * pb);
+      if (elect_one()) commit(o_done + 8 * pb);
       __syncwarp();
     };
     int j = 0, kq = 0, prev_k = 0;
     bool prev_first = false;
-    for (int L = blockIdx.x; L < p.n_items && ok; L += gridDim.x) {
-      const PrefillItem it = prefill_item(p, L);
+    for (int L = item0; L < p.n_items && ok; L += istride) {
+      const PrefillItem it = prefill_item(p, L, (int)cr);
       if (it.ntiles == 0) continue;
       const int qb = kq % T::NQ;
       for (int i = 0; i < it.ntiles && ok; ++i, ++j) {
         const int sb = j & 1;
         if (i == 0 && j > 0) pv(j - 1, prev_first, prev_k);  // finish the previous item
         if (i == 0) {
-          ok = ok && mbar_wait_warp(q_full + 8 * qb, (kq / T::NQ) & 1, abort_flag, p.timeout_ns, 26);
+          ok = ok && waitw(q_full + 8 * qb, (kq / T::NQ) & 1, abort_flag, 26);
           if (!ok) break;
         }
         // S buffer sb last held P(j - 2): PV(j - 2) must have completed
-        if (j >= 2) ok = mbar_wait_warp(o_done + 8 * sb, ((j - 2) >> 1) & 1, abort_flag, p.timeout_ns, 27);
+        if (j >= 2) ok = waitw(o_done + 8 * sb, ((j - 2) >> 1) & 1, abort_flag, 27);
         if (!ok) break;
         tc_fence_after();
-        for (int c = 0; c < T::KCH && ok; c += T::GCH) {
-          ok = mbar_wait_warp(full_bar(grp), ph, abort_flag, p.timeout_ns, 28);
+        for (int c = 0; c < T::KCH && ok; c += T::K_GCH) {
+          ok = waitw(full_bar(grp), ph, abort_flag, 28);
           if (!ok) break;
           tc_fence_after();
           if (elect_one()) {
-            // A = Q chunks c, c+1; B = the group's two K chunks: both K-major,
-            // 128-byte swizzle, 8-row groups 1024 bytes apart, 32 bytes per K step
+            // A = Q chunks c.., B = the group's K chunks: both K-major, 128-byte
+            // swizzle, 8-row groups 1024 bytes apart, 32 bytes per K step.  A
+            // K chunk of the group is K_ROWS x 128 bytes (pairs: this CTA's 64
+            // of the tile's 128 keys, the pair MMA taking N = 128 from both).
             const uint64_t ad0 = umma_sdesc(qs + qb * T::Q_BYTES + c * T::SLOT, 16, 1024, SMEM_SW128);
             const uint64_t bd0 = umma_sdesc(ring + grp * T::GBYTES, 16, 1024, SMEM_SW128);
             const uint32_t d = tmem + T::TMEM_S + sb * 128;
-            umma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
+            mma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
             // the second chunk of an odd count's last pair is padding: skipped
-            const int nks = c + 1 < T::KCH ? 8 : 4;
+            const int nks = c + T::K_GCH <= T::KCH ? 4 * T::K_GCH : 4 * (T::KCH - c);
 #pragma unroll
-            for (int ks = 1; ks < 8; ++ks) {
-              const uint64_t off = (uint64_t)((ks >> 2) * (T::SLOT >> 4) + (ks & 3) * 2);
-              if (ks < nks) umma_ss(d, ad0 + off, bd0 + off, idS, 1u);
+            for (int ks = 1; ks < 4 * T::K_GCH; ++ks) {
+              const uint64_t aoff = (uint64_t)((ks >> 2) * (T::SLOT >> 4) + (ks & 3) * 2);
+              const uint64_t boff = (uint64_t)((ks >> 2) * (T::K_ROWS * 128 >> 4) + (ks & 3) * 2);
+              if (ks < nks) mma_ss(d, ad0 + aoff, bd0 + boff, idS, 1u);
             }
-            umma_commit(empty_bar(grp));
+            commit(empty_bar(grp));
           }
           __syncwarp();
           if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
         }
         if (!ok) break;
         if (elect_one()) {
-          umma_commit(s_full + 8 * sb);
-          if (i == it.ntiles - 1) umma_commit(q_free + 8 * qb);  // this item's Q is free
+          commit(s_full + 8 * sb);
+          if (i == it.ntiles - 1) commit(q_free + 8 * qb);  // this item's Q is free
         }
         __syncwarp();
         if (i > 0) pv(j - 1, prev_first, prev_k);
@@ -361,12 +423,16 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     auto group_and = [&](bool v) { return named_bar_and(1 + wq, 32 * SPLIT, v); };
     volatile int own_abort = 0;
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
-      return mbar_wait_warp(bar, parity, &own_abort, p.timeout_ns, id);
+      return waitw(bar, parity, &own_abort, id);
+    };
+    // pairs: the P and O handshakes are counted on CTA 0's barriers
+    auto arrive_lead = [&](uint32_t bar) {
+      if constexpr (PAIR) mbar_arrive_remote(mapa_shared(bar, 0)); else mbar_arrive(bar);
     };
     bool ok = true;
     int j = 0;
-    for (int L = blockIdx.x; L < p.n_items; L += gridDim.x) {
-      const PrefillItem it = prefill_item(p, L);
+    for (int L = item0; L < p.n_items; L += istride) {
+      const PrefillItem it = prefill_item(p, L, (int)cr);
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
       lim = max(0, min(it.skv, lim));
@@ -465,7 +531,7 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
         l += ((lc[0] + lc[1]) + (lc[2] + lc[3])) + ((lc[4] + lc[5]) + (lc[6] + lc[7]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full + 8 * sb);
+        arrive_lead(p_full + 8 * sb);
       }
 
       // ------------------------------------------------------ epilogue
@@ -510,7 +576,7 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
       }
       if (it.ntiles > 0) {  // O may now be overwritten by the next item's PV
         tc_fence_before();
-        mbar_arrive(o_free);
+        arrive_lead(o_free);
       }
       if (qd == 0 && it.part == 0 && p.lse && qi < p.Sq)
         p.lse[((int64_t)it.b * p.Hq + it.h) * p.Sq + qi] =
@@ -518,13 +584,37 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     }
     if (!ok) *abort_flag = 1;
   }
-  abort_tail(abort_flag, warp, drain);
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, T::TMEM_COLS);
+  if constexpr (PAIR) {
+    // After a give-up in either CTA, CTA 0's issued pair MMAs (reading both
+    // CTAs' shared memory and TMEM) and each CTA's copies must land before
+    // the pair leaves.
+    __syncthreads();
+    if (*abort_flag) {
+      if (warp == 1 && cr == 0) {
+        if (elect_one()) umma_commit_pair(drain);
+        __syncwarp();
+        volatile int never = 0;
+        mbar_wait_warp(drain, 0, &never, 1000000ull, 29);
+      }
+      if (threadIdx.x == 0) {
+        const uint64_t t0n = global_timer_ns();
+        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
+      }
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc_pair(tmem, T::TMEM_COLS);
+    }
+  } else {
+    abort_tail(abort_flag, warp, drain);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, T::TMEM_COLS);
+    }
   }
 }
 
