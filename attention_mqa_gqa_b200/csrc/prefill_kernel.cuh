@@ -105,12 +105,13 @@ struct PrefillTraits {
   static constexpr int QCH = (KCH + 1) & ~1;     // chunk slots per Q row: pairs, the
                                                  // last one zero-filled if KCH is odd
   static constexpr int VCH = DVH / 64;           // V chunks per key tile (this item's columns)
-  // softmax threads per q row: 2 at d_k = 512 (bound by copies and MMA),
-  // 4 otherwise (bound by the softmax's instruction issue: more warps hide
-  // more latency)
-  static constexpr int SPLIT = (DK >= 512) ? 2 : 4;
+  // softmax threads per q row: 4 (the softmax is bound by instruction
+  // issue: more warps hide more latency), except 2 at d_k = 512 on one SM,
+  // where shared memory has no room for the larger exchange buffers
+  static constexpr int SPLIT = (DK >= 512 && !PAIR) ? 2 : 4;
   static constexpr int NQ = (DK >= 512 || QCH > 2) ? 1 : 2;  // Q buffers
-  static constexpr int RING = (DK >= 512) ? 6 : 8;            // 16 KB chunk slots
+  // 16 KB chunk slots (pairs copy half as much per SM: a shallower ring)
+  static constexpr int RING = PAIR ? 4 : (DK >= 512 ? 6 : 8);
   static constexpr int SLOT = 16384;
   // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
   // copies of a single 16 KB chunk cap a CTA's stream well below what the
@@ -124,7 +125,7 @@ struct PrefillTraits {
   // row exchange buffers float [XR][SPLIT][128]: two rounds alternate with
   // the tile (one barrier per exchange); at d_k = 512 shared memory has room
   // for one round only, which then takes a second barrier
-  static constexpr int XR = (DK >= 512) ? 1 : 2;
+  static constexpr int XR = (DK >= 512 && !PAIR) ? 1 : 2;
   static constexpr int OFF_XCH = OFF_RING + RING * SLOT;
   static constexpr int OFF_FLAGS = OFF_XCH + XR * SPLIT * 128 * 4;  // abort, tmem base
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
