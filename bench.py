@@ -437,18 +437,19 @@ def reference_arm(args, world, rank):
     from oracle import c_oracle
 
     c_oracle.build()
+    steps = args.steps if args.steps else 3
     for _ in range(args.warmup):
         run_oracle(w, inp, n)
     t = 0.0
-    for _ in range(args.steps):
+    for _ in range(steps):
         t += run_oracle(w, inp, n)
-    val = cpu_value(w, inp, n, t / args.steps)
+    val = cpu_value(w, inp, n, t / steps)
     metric, unit, hib = metric_of(w)
     cores = os.cpu_count() or 1
     sample = f"first {n} of {w.B} sequences, all {w.Hq} heads, per step"
     line = {"impl": "reference", "metric": f"{w.name}_{metric}", "value": round(val, 4),
-            "unit": unit, "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": hib,
+            "unit": unit, "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(t / steps * 1e3, 3), "higher_is_better": hib,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, inp, "host cores"),
             "cpu_baseline": {"value": round(val, 4), "unit": unit, "cores": cores,
