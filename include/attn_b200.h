@@ -17,7 +17,9 @@
  * Absorbed MLA decode ("Full 路线" section 4.3: W_UK folded into the query,
  * the cache holds rows [c_kv (512) | k_pe (64)]) is the same call with
  * d_k = 576, d_v = 512, Hkv = 1 and v pointing at the same rows as k (the
- * first 512 columns): the kernel then loads each cached row once.
+ * first 512 columns): each cached row then comes from DRAM about once (its
+ * first 512 columns are read again as V from L2), and all query heads of a
+ * sequence share it (pairs of SMs, 128 heads per pair).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
