@@ -176,6 +176,47 @@ def split_combine(o_parts, lse_parts):
     return out, L
 
 
+def topk_attention_fwd(q, k, v, skv_lens, idx, n_sel, scale: float):
+    """Attention of each query over a selected subset of its sequence's keys.
+
+    "带你了解Attention,从MHA到DeepSeek" section 5.1 (DSA): an indexer picks the
+    top-k cached entries per new token and attention is computed over those
+    entries only.  The indexer itself is not modelled: the selection is an
+    input.  For sequence b the selected keys are the positions
+    idx[b, t], t < n_sel[b]; every query row i of every head h of b gets
+
+        out = sum_t exp(s_t - m) v[b, h//G, idx[b,t]] / sum_t exp(s_t - m),
+        s_t = scale * q[b,h,i] . k[b, h//G, idx[b,t]],  lse = m + log sum_t exp(s_t - m)
+
+    (one selection per sequence, shared by its query rows and heads; no
+    causal mask beyond the selection).  A position listed twice counts twice.
+    n_sel[b] == 0 gives out 0, lse -inf.  Positions outside [0, skv[b]) raise.
+    Returns (out [B, Hq, Sq, d_v], lse [B, Hq, Sq]) in float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    idx = np.asarray(idx.tolist() if hasattr(idx, "tolist") else idx, dtype=np.int64)
+    B, Hq, Sq, _ = q.shape
+    Hkv, d_v = k.shape[1], v.shape[-1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, Sq, d_v))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    for b in range(B):
+        n = int(n_sel[b])
+        if n == 0:
+            continue
+        sel = idx[b, :n]
+        if sel.min() < 0 or sel.max() >= int(skv_lens[b]):
+            raise ValueError(f"sequence {b}: a selected position lies outside [0, skv)")
+        for h in range(Hq):
+            kh, vh = k[b, h // G][sel], v[b, h // G][sel]  # [n, d]
+            s = scale * (q[b, h] @ kh.T)  # [Sq, n]
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            out[b, h] = (e @ vh) / l
+            lse[b, h] = (m + np.log(l))[:, 0]
+    return out, lse
+
+
 # --------------------------------------------------------------------------
 # MLA: naive reconstruction versus attention over the absorbed latent rows.
 # "Full 路线" sections 4.2-4.3; "GQA和MLA详解" section 3 (matrix absorption:

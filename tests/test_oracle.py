@@ -315,3 +315,89 @@ def test_byte_model_matches_printed_tables():
     mq = g["mqa_cache_fraction"]
     assert npo.kv_bytes_per_token("mqa", d_h=512) / npo.kv_bytes_per_token(
         "mha", H=mq["query_heads"], d_h=512) == mq["fraction"]
+
+
+# ------------------------------------------------------- top-k (DSA) pins
+
+def _topk_case(seed, B=3, Hq=8, Hkv=2, Sq=1, S=40, d=16, dv=12):
+    q = rnd((B, Hq, Sq, d), seed)
+    k = rnd((B, Hkv, S, d), seed + 1)
+    v = rnd((B, Hkv, S, dv), seed + 2)
+    return q, k, v
+
+
+def test_topk_matches_sdpa_on_library_gathered_rows():
+    """Attention over the selected keys equals torch SDPA (fp64, enable_gqa)
+    on K/V rows picked by torch.index_select, per sequence ("带你了解Attention"
+    section 5.1: attention runs over the top-k entries only)."""
+    q, k, v = _topk_case(60, Sq=3)
+    skv = [40, 25, 9]
+    g = np.random.default_rng(61)
+    n_sel = [7, 25, 1]
+    idx = np.zeros((3, 25), dtype=np.int64)
+    for b in range(3):
+        idx[b, :n_sel[b]] = g.choice(skv[b], n_sel[b], replace=False)
+    out, lse = npo.topk_attention_fwd(q, k, v, skv, idx, n_sel, 0.4)
+    for b in range(3):
+        sel = torch.from_numpy(idx[b, :n_sel[b]])
+        kb = torch.from_numpy(k[b:b + 1]).index_select(2, sel)
+        vb = torch.from_numpy(v[b:b + 1]).index_select(2, sel)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b:b + 1]), kb, vb, scale=0.4, enable_gqa=True).numpy()
+        np.testing.assert_allclose(out[b:b + 1], ref, rtol=1e-12, atol=1e-13)
+        s = 0.4 * torch.from_numpy(q[b]) @ kb[0].repeat_interleave(4, dim=0).transpose(-1, -2)
+        np.testing.assert_allclose(lse[b], torch.logsumexp(s, dim=-1).numpy(), rtol=1e-12)
+
+
+def test_topk_all_positions_is_dense_decode():
+    """Selecting every position of a sequence is ordinary decode attention
+    (pinned above against SDPA)."""
+    q, k, v = _topk_case(62)
+    skv = [40, 3, 17]
+    idx = np.zeros((3, 40), dtype=np.int64)
+    for b, L in enumerate(skv):
+        idx[b, :L] = np.arange(L)
+    out, lse = npo.topk_attention_fwd(q, k, v, skv, idx, skv, 0.3)
+    ref_o, ref_l = npo.attention_fwd(q, k, v, skv, 0.3, True)
+    np.testing.assert_allclose(out, ref_o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, ref_l, rtol=1e-12, atol=1e-13)
+
+
+def test_topk_selection_order_and_union():
+    """The order of the selected positions does not matter, and attention over
+    a union of two disjoint selections is the LSE-weighted merge of the two."""
+    q, k, v = _topk_case(63, B=1)
+    idx = np.array([[5, 31, 2, 17, 39, 0, 22, 8]])
+    a_o, a_l = npo.topk_attention_fwd(q, k, v, [40], idx, [8], 0.5)
+    b_o, b_l = npo.topk_attention_fwd(q, k, v, [40], idx[:, ::-1].copy(), [8], 0.5)
+    np.testing.assert_allclose(a_o, b_o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(a_l, b_l, rtol=1e-13, atol=1e-14)
+    p_o, p_l = npo.topk_attention_fwd(q, k, v, [40], idx[:, :3].copy(), [3], 0.5)
+    r_o, r_l = npo.topk_attention_fwd(q, k, v, [40], idx[:, 3:].copy(), [5], 0.5)
+    m_o, m_l = npo.split_combine(np.stack([p_o, r_o]), np.stack([p_l, r_l]))
+    np.testing.assert_allclose(m_o, a_o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(m_l, a_l, rtol=1e-13, atol=1e-14)
+
+
+def test_topk_single_repeated_and_empty():
+    """One selected key: out is its value row, lse its score.  The same key
+    listed twice: the same row, lse + ln 2.  Nothing selected: 0 and -inf."""
+    q, k, v = _topk_case(64, B=3, Hq=2, Hkv=1)
+    idx = np.array([[13, 0], [13, 13], [0, 0]])
+    out, lse = npo.topk_attention_fwd(q, k, v, [40, 40, 40], idx, [1, 2, 0], 0.25)
+    for h in range(2):
+        s = 0.25 * float(q[0, h, 0] @ k[0, 0, 13])
+        np.testing.assert_array_equal(out[0, h, 0], v[0, 0, 13])
+        assert abs(lse[0, h, 0] - s) < 1e-13
+        s1 = 0.25 * float(q[1, h, 0] @ k[1, 0, 13])
+        np.testing.assert_allclose(out[1, h, 0], v[1, 0, 13], rtol=1e-15, atol=1e-15)
+        assert abs(lse[1, h, 0] - (s1 + math.log(2))) < 1e-13
+    assert (out[2] == 0).all() and np.isneginf(lse[2]).all()
+
+
+def test_topk_rejects_positions_outside_the_sequence():
+    q, k, v = _topk_case(65, B=1)
+    with pytest.raises(ValueError):
+        npo.topk_attention_fwd(q, k, v, [10], np.array([[3, 10]]), [2], 0.5)
+    with pytest.raises(ValueError):
+        npo.topk_attention_fwd(q, k, v, [10], np.array([[-1, 2]]), [2], 0.5)
