@@ -339,22 +339,31 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       };
       PieceWalker w = walker();
       int b, kvh, t0, n;
-      int pv_tok = -1, pv_kvh = 0, pv_b = 0;  // tile whose V is still to be loaded
+      int pv_tok = 0, pv_kvh = 0, pv_b = 0;  // tile whose V is still to be loaded
+      bool have_prev = false;
       auto load_v = [&]() {
         for (int c = 0; c < T::VCH; c += T::GCH) load(&tmV, c, pv_tok, pv_kvh, pv_b);
       };
       while (ok && w.next(b, kvh, t0, n)) {
+        // A sequence's partial last tile is read as the 128 rows that end at
+        // its last key (the rows before the tile are masked): every row read
+        // is then a key of the sequence, so whatever the cache holds past
+        // skv -- unwritten memory, NaN -- never meets a zero weight in P.V.
+        // A sequence shorter than the tile starts at a negative row, which
+        // the copy fills with zeros.
+        const int last_win = p.skv[b] - T::TILE;
         for (int i = 0; i < n && ok; ++i) {
-          const int tok = (t0 + i) * T::TILE;
-          if (i == 0 && pv_tok >= 0) load_v();  // finish the previous piece first
+          const int tok = min((t0 + i) * T::TILE, last_win);
+          if (i == 0 && have_prev) load_v();  // finish the previous piece first
           for (int c = 0; c < T::KCH; c += T::GCH) load(&tmK, c, tok, kvh, b);
           if (i > 0) load_v();
           pv_tok = tok;
           pv_kvh = kvh;
           pv_b = b;
+          have_prev = true;
         }
       }
-      if (pv_tok >= 0) load_v();
+      if (have_prev) load_v();
     } else if (warp == 0 && lane == 1) {
       // ------------------------------------------------ producer: Q^T per piece
       tma_prefetch_desc(&tmQ);
@@ -513,10 +522,13 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
           // Column c holds query qi = c % Sq (Sq a power of two), which sees
           // keys <= skv_b - Sq + qi under the causal mask (bottom-right
           // alignment) and keys < skv_b otherwise; with kq = key - (skv_b - Sq)
-          // the causal test is kq <= qi.
-          const int key = (t0 + i) * T::TILE + row;
+          // the causal test is kq <= qi.  The rows of a partial last tile
+          // are the 128 keys ending at skv_b; those before the tile's start
+          // belong to the previous tile and are masked here.
+          const int tile0 = (t0 + i) * T::TILE;
+          const int key = min(tile0, skv_b - T::TILE) + row;
           const int kq = key - (skv_b - p.Sq);
-          const bool in_seq = key < skv_b;
+          const bool in_seq = key >= tile0;
           const int sq_mask = p.Sq - 1;
           // This thread's HH scores of its key (scaled to log2 units, masked),
           // read from TMEM twice: for the maxima and again for the weights,
@@ -526,7 +538,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < HH; ++e) {
-              const bool vis = p.causal ? kq <= ((h0l + e) & sq_mask) : in_seq;
+              const bool vis = in_seq && (!p.causal || kq <= ((h0l + e) & sq_mask));
               x[e] = vis ? x[e] * p.scale_log2 : -INFINITY;
             }
           };

@@ -221,25 +221,31 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
       };
       PieceWalker w = walker();
       int b, kvh, t0, n;
-      int pv_t = -1, pv_kvh = 0, pv_b = 0;  // pair tile whose V is still to be loaded
+      int pv_row = 0, pv_kvh = 0, pv_b = 0;  // pair tile whose V is still to be loaded
+      bool have_prev = false;
       // V block m of this CTA = chunks 4m + 2cr, +1, for the tile's 256 keys
       auto load_v = [&]() {
         for (int m = 0; m < 2; ++m)
           for (int h = 0; h < 2; ++h)
-            load(&tmV, 4 * m + 2 * (int)cr, pv_t * 256 + 128 * h, pv_kvh, pv_b, pol_v);
+            load(&tmV, 4 * m + 2 * (int)cr, pv_row + 128 * h, pv_kvh, pv_b, pol_v);
       };
       while (ok && w.next(b, kvh, t0, n)) {
+        // a partial last pair tile is read as the 256 rows ending at the
+        // sequence's last key (earlier rows masked), so no row past skv --
+        // possibly unwritten memory -- is read; a negative start reads zeros
+        const int last_win = p.skv[b] - 256;
         for (int i = 0; i < n && ok; ++i) {
-          const int t = t0 + i;
-          if (i == 0 && pv_t >= 0) load_v();  // finish the previous piece first
-          for (int c = 0; c < T::KCH; c += 2) load(&tmK, c, t * 256 + 128 * (int)cr, kvh, b, pol_k);
+          const int row0 = min((t0 + i) * 256, last_win);
+          if (i == 0 && have_prev) load_v();  // finish the previous piece first
+          for (int c = 0; c < T::KCH; c += 2) load(&tmK, c, row0 + 128 * (int)cr, kvh, b, pol_k);
           if (i > 0) load_v();
-          pv_t = t;
+          pv_row = row0;
           pv_kvh = kvh;
           pv_b = b;
+          have_prev = true;
         }
       }
-      if (pv_t >= 0) load_v();
+      if (have_prev) load_v();
     } else if (warp == 0 && lane == 1) {
       // ------------------------------------------------ producer: Q^T half per piece
       tma_prefetch_desc(&tmQ);
@@ -390,7 +396,10 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
           ok = wait(s_full + 8 * sb, (j >> 1) & 1, 51);
           if (!ok) break;
           tc_fence_after();
-          const bool valid = (t0 + i) * 256 + (int)cr * T::TILE + row < skv_b;
+          // rows of a partial last tile end at skv_b; those before the
+          // tile's start belong to the previous tile
+          const int tile0 = (t0 + i) * 256;
+          const bool valid = min(tile0, skv_b - 256) + (int)cr * T::TILE + row >= tile0;
           const uint32_t s_col = tmem + lane_base + T::TMEM_S + sb * NH + h0l;
 
           // this CTA's per-head maximum over its 128 keys

@@ -251,6 +251,10 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     };
     bool have_prev = false;
     int pv_tok = 0, pv_kvh = 0, pv_b = 0, pv_ch = 0;  // tile whose V is still to load
+    // A partial last key tile is read as the KT rows ending at the
+    // sequence's last key (the rows before the tile are masked), so no row
+    // past skv -- possibly unwritten memory -- enters P.V; a negative start
+    // reads zeros.
     auto load_v = [&]() {
       for (int c = 0; c < T::V_CH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
     };
@@ -258,10 +262,11 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
       const PrefillItem it = prefill_item(p, L, (int)cr);
       for (int j = 0; j < it.ntiles && ok; ++j) {
         if (j == 0 && have_prev) load_v();  // finish the previous item first
+        const int row0 = min(j * T::KT, it.skv - T::KT);
         for (int c = 0; c < T::KCH; c += T::K_GCH)
-          load(&tmK, c, j * T::KT + (int)cr * T::K_ROWS, it.kvh, it.b);
+          load(&tmK, c, row0 + (int)cr * T::K_ROWS, it.kvh, it.b);
         if (j > 0) load_v();
-        pv_tok = j * T::KT;
+        pv_tok = row0;
         pv_kvh = it.kvh;
         pv_b = it.b;
         // pairs: this CTA's half of the part's DVH columns
@@ -450,14 +455,18 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
           tmem_ld<KS>(tmem + lane_base + T::TMEM_S + sb * 128 + qd * KS, s);
           tmem_wait_ld();
 
-          const int kb = i * T::KT + qd * KS;
           // Keys at or past `lim` are invisible to this row; only tiles that
-          // straddle `lim` need the mask.  The maximum is taken on the raw
-          // scores (scale > 0) in 8 independent chains, then scaled once.
-          if (kb + KS > lim) {
+          // straddle `lim` need the mask.  A partial last tile holds the KT
+          // keys ending at skv; its keys below the tile start t0k belong to
+          // the previous tile and are masked too.  The maximum is taken on
+          // the raw scores (scale > 0) in 8 independent chains, then scaled
+          // once.
+          const int t0k = i * T::KT;
+          const int kb = min(t0k, it.skv - T::KT) + qd * KS;
+          if (kb + KS > lim || kb < t0k) {
 #pragma unroll
             for (int c = 0; c < KS; ++c)
-              if (kb + c >= lim) s[c] = -INFINITY;
+              if (kb + c >= lim || kb + c < t0k) s[c] = -INFINITY;
           }
           float mc[8];
 #pragma unroll

@@ -26,10 +26,24 @@ def _built():
         pytest.skip("no CUDA device")
 
 
+def _poison_past_length(inp):
+    """Set every cache row at or past its sequence's length to NaN.  Those
+    rows are not part of the problem (a cache allocated for max_skv keys
+    holds whatever memory had there), so the result must not change."""
+    for b, L in enumerate(inp["skv"].tolist()):
+        if "cache" in inp:
+            inp["cache"][b, L:] = float("nan")
+        else:
+            inp["k"][b, :, L:] = float("nan")
+            inp["v"][b, :, L:] = float("nan")
+
+
 def _case(B, Hq, Hkv, Sq, skv, dk, dv, dtype=torch.bfloat16, causal=True, mla=False, seed=0,
-          max_skv=None, scale=None):
+          max_skv=None, scale=None, poison=False):
     w, inp = wl.make_case(B, Hq, Hkv, Sq, skv, dk, dv, dtype=dtype, causal=causal, mla=mla,
                           seed=seed, max_skv=max_skv, scale=scale)
+    if poison:
+        _poison_past_length(inp)
     dev = to_device(inp)
     out, lse = run_gpu(w, dev)
     ref_o, ref_l = oracle_full(w, inp)
@@ -148,6 +162,32 @@ def test_prefill_mqa_tiny_workload():
     out, lse = run_gpu(w, to_device(inp))
     ref_o, ref_l = oracle_full(w, inp)
     compare(out, lse, ref_o, ref_l, w.name)
+
+
+# --------------------------------------- cache rows past a sequence's end
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,skv,max_skv,dk,dv,mla", [
+    (3, 16, 2, 1, [1, 129, 700], 1024, 128, 128, False),     # GQA decode
+    (3, 16, 1, 1, [1, 300, 2049], 2100, 512, 512, False),    # MQA d=512 decode
+    (3, 128, 1, 1, [1, 200, 1500], 1600, 576, 512, True),    # MLA pair decode
+    (2, 16, 2, 4, [1000, 3], 1100, 128, 128, False),         # extend, Sq = 4
+])
+def test_decode_ignores_rows_past_length(B, Hq, Hkv, Sq, skv, max_skv, dk, dv, mla):
+    """NaN in every cache row at or past skv[b] (as in a cache allocated for
+    max_skv keys and filled as it grows) must not reach the output."""
+    _case(B, Hq, Hkv, Sq, skv, dk, dv, mla=mla, seed=80 + Sq, max_skv=max_skv, poison=True,
+          scale=1 / math.sqrt(192) if mla else None)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,skv,max_skv,dk,dv", [
+    (2, 8, 1, 150, [300, 100], 320, 128, 128),     # d=128, varlen, bottom-right
+    (2, 16, 1, 129, [129, 129], 200, 512, 512),    # d=512, SM pairs (even G)
+    (1, 3, 1, 129, [150], 256, 512, 512),          # d=512, one CTA per tile (odd G)
+    (1, 4, 2, 129, [200], 256, 192, 128),          # expanded MLA, d_k 192 / d_v 128
+    (1, 4, 2, 100, [100], 256, 128, 128),          # shorter than one key tile
+])
+def test_prefill_ignores_rows_past_length(B, Hq, Hkv, Sq, skv, max_skv, dk, dv):
+    _case(B, Hq, Hkv, Sq, skv, dk, dv, seed=90 + Sq, max_skv=max_skv, poison=True)
 
 
 # ------------------------------------------------------------- determinism
