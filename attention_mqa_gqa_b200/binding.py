@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
 
 (ATTN_OK, ATTN_EINVAL, ATTN_EUNSUPPORTED, ATTN_EWORKSPACE, ATTN_ECUDA, ATTN_ETIMEOUT,
- ATTN_EOVERFLOW) = range(7)
+ ATTN_EOVERFLOW, ATTN_EINDEX) = range(8)
 ATTN_BF16, ATTN_FP16 = 0, 1
 
 
@@ -43,7 +43,8 @@ class AttnError(RuntimeError):
 # Every symbol include/attn_b200.h declares (checked by the CPU test suite).
 EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
            "attn_decode_combine", "attn_fwd_noalloc", "attn_last_device_error", "attn_status_str",
-           "attn_version", "attn_set_wait_timeout_ns", "attn_cache_append")
+           "attn_version", "attn_set_wait_timeout_ns", "attn_cache_append",
+           "attn_gather_rows")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in the header
 
 _lib = None
@@ -75,6 +76,9 @@ def load(path: str | None = None):
     lib.attn_cache_append.restype = i32
     lib.attn_cache_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, Strides,
                                       Strides, Strides, Strides, vp]
+    lib.attn_gather_rows.restype = i32
+    lib.attn_gather_rows.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, Strides,
+                                     Strides, i64, vp]
     lib.attn_set_wait_timeout_ns.restype = ctypes.c_uint64
     lib.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.attn_last_device_error.restype = i32
@@ -213,6 +217,31 @@ def cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor | None, k_new: tor
         raise AttnError(rc, "attn_cache_append")
 
 
+def gather_rows(src: torch.Tensor, dst: torch.Tensor, idx: torch.Tensor, n_sel: torch.Tensor,
+                skv: torch.Tensor, dst_len: torch.Tensor,
+                stream: torch.cuda.Stream | None = None) -> None:
+    """attn_gather_rows: dst[b, h, t] = src[b, h, idx[b, t]] for t < n_sel[b],
+    dst_len[b] = n_sel[b] (device-side).  src [B, H, S, d] and dst
+    [B, H, topk, d] (views allowed, last dim contiguous); idx int32
+    [B, >= topk] (last dim contiguous); n_sel, skv, dst_len int32 [B]."""
+    B, H, topk, d = dst.shape
+    for t in (idx, n_sel, skv, dst_len):
+        if t.dtype != torch.int32:
+            raise TypeError("idx, n_sel, skv and dst_len must be int32")
+    if idx.dim() != 2 or idx.stride(1) != 1 or not n_sel.is_contiguous() \
+            or not skv.is_contiguous() or not dst_len.is_contiguous():
+        raise ValueError("idx rows and n_sel/skv/dst_len must be contiguous")
+    if src.dtype != dst.dtype:
+        raise TypeError("src and dst must have the same element type")
+    st = stream if stream is not None else torch.cuda.current_stream(dst.device)
+    rc = load().attn_gather_rows(src.data_ptr(), dst.data_ptr(), idx.data_ptr(), n_sel.data_ptr(),
+                                 skv.data_ptr(), dst_len.data_ptr(), B, H, topk, d,
+                                 dtype_code(dst.dtype), _strides4(src), _strides4(dst),
+                                 idx.stride(0), st.cuda_stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_gather_rows")
+
+
 def set_wait_timeout_ns(ns: int) -> int:
     """Bound every device-side wait of later launches (0 = default 2 s);
     returns the previous bound.  Diagnostic only (see the header)."""
@@ -230,4 +259,38 @@ def attention(q, k, v, skv, max_skv, scale, causal=True, with_lse=True, workspac
         n = workspace_bytes(B, Hq, k.shape[1], Sq, int(max_skv), q.shape[-1], d_v)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
     attn_fwd(q, k, v, out, skv, max_skv, scale, causal, lse, workspace, stream)
+    return out, lse
+
+
+def topk_attention(q, k_cache, v_cache, idx, n_sel, skv, scale, d_v=None, with_lse=True,
+                   scratch=None, stream=None):
+    """Sparse (top-k) decode: attn_gather_rows copies the selected rows of the
+    caches into scratch caches of topk = idx.shape[1] rows, then attn_fwd
+    attends over them, both on one stream.  k_cache/v_cache [B, Hkv, S, d];
+    for an absorbed-MLA latent cache pass v_cache=None and d_v (the value
+    rows are the first d_v columns of the gathered rows).  ``scratch`` is an
+    optional dict of preallocated device tensors (keys k, v, len, ws) reused
+    between calls.  Returns (out, lse)."""
+    B, Hkv, _, d_k = k_cache.shape
+    topk = idx.shape[1]
+    latent = v_cache is None
+    if latent and d_v is None:
+        raise ValueError("d_v is required for a latent (MLA) cache")
+    d_v = d_v if latent else v_cache.shape[-1]
+    sc = scratch if scratch is not None else {}
+    if "k" not in sc:
+        sc["k"] = torch.empty(B, Hkv, topk, d_k, dtype=k_cache.dtype, device=k_cache.device)
+        sc["v"] = None if latent else torch.empty(B, Hkv, topk, d_v, dtype=k_cache.dtype,
+                                                  device=k_cache.device)
+        sc["len"] = torch.empty(B, dtype=torch.int32, device=k_cache.device)
+        n = workspace_bytes(B, q.shape[1], Hkv, q.shape[2], topk, d_k, d_v)
+        sc["ws"] = torch.empty(max(n, 16), dtype=torch.uint8, device=k_cache.device)
+    gather_rows(k_cache, sc["k"], idx, n_sel, skv, sc["len"], stream)
+    if not latent:
+        gather_rows(v_cache, sc["v"], idx, n_sel, skv, sc["len"], stream)
+    v = sc["k"][..., :d_v] if latent else sc["v"]
+    out = torch.empty(B, q.shape[1], q.shape[2], d_v, dtype=q.dtype, device=q.device)
+    lse = (torch.empty(B, q.shape[1], q.shape[2], dtype=torch.float32, device=q.device)
+           if with_lse else None)
+    attn_fwd(q, sc["k"], v, out, sc["len"], topk, scale, True, lse, sc["ws"], stream)
     return out, lse

@@ -16,6 +16,7 @@
 #include "../../include/attn_b200.h"
 #include "decode_kernel.cuh"
 #include "cache_append.cuh"
+#include "gather_rows.cuh"
 #include "mla_pair_kernel.cuh"
 #include "prefill_kernel.cuh"
 
@@ -515,7 +516,8 @@ attn_status_t attn_last_device_error(void* cuda_stream) {
   if (word != 0 && cudaMemcpyToSymbol(attn::g_attn_error, &zero, sizeof(zero)) != cudaSuccess)
     return ATTN_ECUDA;
   if (word & 1u) return ATTN_ETIMEOUT;
-  return word ? ATTN_EOVERFLOW : ATTN_OK;
+  if (word & 2u) return ATTN_EOVERFLOW;
+  return word ? ATTN_EINDEX : ATTN_OK;
 }
 
 const char* attn_status_str(attn_status_t s) {
@@ -527,6 +529,7 @@ const char* attn_status_str(attn_status_t s) {
     case ATTN_ECUDA: return "CUDA error";
     case ATTN_ETIMEOUT: return "device-side wait timed out";
     case ATTN_EOVERFLOW: return "cache full: a sequence already holds max_skv keys";
+    case ATTN_EINDEX: return "a selected position lies outside its sequence";
   }
   return "unknown status";
 }
@@ -573,6 +576,43 @@ attn_status_t attn_cache_append(void* k_cache, void* v_cache, const void* k_new,
   ap.vn_sb = svn.b;
   ap.vn_sh = svn.h;
   attn::cache_append_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(ap);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+attn_status_t attn_gather_rows(const void* src, void* dst, const int32_t* idx,
+                               const int32_t* n_sel, const int32_t* skv_per_seq, int32_t* dst_len,
+                               int B, int H, int topk, int d, attn_dtype_t dtype,
+                               attn_strides_t s_src, attn_strides_t s_dst, int64_t idx_stride,
+                               void* cuda_stream) {
+  if (!src || !dst || !idx || !n_sel || !skv_per_seq || !dst_len) return ATTN_EINVAL;
+  if (B <= 0 || H <= 0 || topk <= 0 || d <= 0 || d % 8 != 0 || idx_stride < topk) return ATTN_EINVAL;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_EINVAL;
+  if (!aligned16(src) || !aligned16(dst) || !strides_ok(s_src) || !strides_ok(s_dst))
+    return ATTN_EINVAL;
+  for (const void* q : {static_cast<const void*>(idx), static_cast<const void*>(n_sel),
+                        static_cast<const void*>(skv_per_seq), static_cast<const void*>(dst_len)})
+    if (reinterpret_cast<uintptr_t>(q) & 3u) return ATTN_EINVAL;
+  if (B > 65535 || H > 65535) return ATTN_EUNSUPPORTED;
+  attn::GatherParams gp{};
+  gp.src = reinterpret_cast<const uint8_t*>(src);
+  gp.dst = reinterpret_cast<uint8_t*>(dst);
+  gp.idx = idx;
+  gp.n_sel = n_sel;
+  gp.skv = skv_per_seq;
+  gp.dst_len = dst_len;
+  gp.B = B;
+  gp.H = H;
+  gp.topk = topk;
+  gp.d = d;
+  gp.s_sb = s_src.b;
+  gp.s_sh = s_src.h;
+  gp.s_ss = s_src.s;
+  gp.d_sb = s_dst.b;
+  gp.d_sh = s_dst.h;
+  gp.d_ss = s_dst.s;
+  gp.i_sb = idx_stride;
+  const dim3 grid((unsigned)((topk + 127) / 128), (unsigned)H, (unsigned)B);
+  attn::gather_rows_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(gp);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 

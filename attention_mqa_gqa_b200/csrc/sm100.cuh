@@ -97,7 +97,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Device error word (one per device, read and cleared by the host).
 // Bit layout: bit 0 = some wait timed out; bit 1 = a cache append found a
-// full sequence; bits 8..15 = id of the first barrier that timed out.
+// full sequence; bit 2 = a row gather met a position outside its sequence;
+// bits 8..15 = id of the first barrier that timed out.
 __device__ unsigned int g_attn_error;
 
 // Bounded wait on phase `parity` of `bar`.  Gives up after `timeout_ns` of

@@ -40,6 +40,7 @@ class Workload:
     scale: float
     mla: bool
     seed: int
+    topk: int = 0  # > 0: attention over at most topk selected positions per sequence
 
     @property
     def G(self) -> int:
@@ -50,7 +51,7 @@ class Workload:
         """Runs on the split-KV decode path and is bound by reading the KV
         cache: one query per sequence, or a few (a power of two up to 16 at
         head dim 128 or 512: extend / speculative-decoding verification)."""
-        if self.Sq == 1:
+        if self.Sq == 1 or self.topk:
             return True
         return (self.d_k in (128, 512) and self.d_k == self.d_v and self.Sq <= 16
                 and self.Sq & (self.Sq - 1) == 0)
@@ -78,6 +79,10 @@ WORKLOADS = {
     # speculative-decoding verify step: 4 queries per sequence against the cache
     "gqa_extend": Workload("gqa_extend", 64, 64, 8, 4, 4096, 4096, 128, 128,
                            torch.bfloat16, True, 1 / math.sqrt(128), False, 6),
+    # DSA-style sparse decode over the absorbed-MLA cache: per sequence 2048
+    # of 16K-48K cached positions are selected (the selection is an input)
+    "mla_topk_decode": Workload("mla_topk_decode", 64, 128, 1, 1, 16384, 49152, 576, 512,
+                                torch.bfloat16, True, 1 / math.sqrt(192), True, 7, topk=2048),
     # MLA prefill in the expanded (MHA) form: 128 heads, q/k head dim 192
     # (128 nope + 64 rope columns, already rotated), v head dim 128
     "mla_prefill": Workload("mla_prefill", 1, 128, 128, 4096, 4096, 4096, 192, 128,
@@ -96,11 +101,28 @@ def _randn_into(t: torch.Tensor, g: torch.Generator, rows_per_chunk: int = 1 << 
         flat[s:e].copy_(torch.randn(e - s, generator=g, dtype=torch.float32))
 
 
+def make_selection(skv, topk: int, g: torch.Generator):
+    """Stand-in for an indexer's top-k choice: per sequence, min(topk, skv[b])
+    distinct positions of [0, skv[b]) drawn uniformly, in ascending order.
+    Returns (idx int32 [B, topk] -- unused slots 0 --, n_sel int32 [B])."""
+    B = len(skv)
+    idx = torch.zeros(B, topk, dtype=torch.int32)
+    n_sel = torch.zeros(B, dtype=torch.int32)
+    for b in range(B):
+        L = int(skv[b])
+        n = min(topk, L)
+        if n:
+            idx[b, :n] = torch.randperm(L, generator=g)[:n].sort().values.to(torch.int32)
+        n_sel[b] = n
+    return idx, n_sel
+
+
 def make_inputs(w: Workload, skv_override=None) -> dict:
     """Draw the inputs of workload ``w`` on the CPU.
 
     Returns a dict with q, k, v (CPU tensors of w.dtype), skv (int32 [B]),
-    max_skv, and for MLA the backing ``cache`` tensor."""
+    max_skv, for MLA the backing ``cache`` tensor, and for a top-k workload
+    the selection ``idx`` (int32 [B, topk]) and ``n_sel`` (int32 [B])."""
     g = torch.Generator().manual_seed(w.seed)
     skv = torch.randint(w.skv_lo, w.skv_hi + 1, (w.B,), generator=g, dtype=torch.int64)
     if skv_override is not None:
@@ -122,6 +144,8 @@ def make_inputs(w: Workload, skv_override=None) -> dict:
         v = torch.empty(w.B, w.Hkv, S, w.d_v, dtype=w.dtype)
         _randn_into(v, g)
         out["k"], out["v"] = k, v
+    if w.topk:
+        out["idx"], out["n_sel"] = make_selection(skv.tolist(), w.topk, g)
     return out
 
 

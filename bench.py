@@ -47,15 +47,23 @@ KERNEL_SOURCES = {
     "mla_pair_kernel": [_CSRC + "sm100.cuh", _CSRC + "decode_kernel.cuh", _CSRC + "mla_pair_kernel.cuh",
                         _CSRC + "attn_api.cu"],
     "prefill_kernel": [_CSRC + "sm100.cuh", _CSRC + "prefill_kernel.cuh", _CSRC + "attn_api.cu"],
+    "gather_rows_kernel": [_CSRC + "sm100.cuh", _CSRC + "gather_rows.cuh", _CSRC + "attn_api.cu"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 # ----------------------------------------------------------------- accounting
 
+def keys_of(w, inp):
+    """Keys each sequence attends to: its length, or for a top-k workload
+    the number of selected positions."""
+    return inp["n_sel"] if w.topk else inp["skv"]
+
+
 def kv_bytes(w, skv) -> int:
     """Cached K/V bytes one decode step must read: every key row of every
-    sequence once (MLA: the 576-wide row once, V aliases its first 512)."""
+    sequence once (MLA: the 576-wide row once, V aliases its first 512).
+    For a top-k workload pass the selected counts: the selected rows once."""
     n = int(sum(int(x) for x in skv))
     el = 2
     if w.mla:
@@ -195,6 +203,19 @@ class GpuRunner:
             self.k = inp["k"].to(device)
             self.v = inp["v"].to(device)
         self.skv = inp["skv"].to(device)
+        self.topk = w.topk
+        if self.topk:
+            # the step: gather the selected rows of the latent cache into a
+            # dense cache of topk rows, then the split decode over it
+            if not w.mla:
+                raise ValueError("top-k workloads are defined on the MLA latent cache")
+            self.src_k, self.src_skv = self.k, self.skv
+            self.idx = inp["idx"].to(device)
+            self.n_sel = inp["n_sel"].to(device)
+            sel = torch.empty(w.B, 1, self.topk, w.d_k, dtype=w.dtype, device=device)
+            self.k, self.v = sel, sel[..., : w.d_v]
+            self.skv = torch.empty(w.B, dtype=torch.int32, device=device)
+            self.max_skv = self.topk
         self.out = torch.empty(w.B, w.Hq, w.Sq, w.d_v, dtype=w.dtype, device=device)
         self.lse = torch.empty(w.B, w.Hq, w.Sq, dtype=torch.float32, device=device)
         nws = binding.workspace_bytes(w.B, w.Hq, w.Hkv, w.Sq, self.max_skv, w.d_k, w.d_v)
@@ -215,7 +236,15 @@ class GpuRunner:
                           self.stream.cuda_stream)
         return self._args
 
+    def gather(self):
+        self.b.gather_rows(self.src_k, self.k, self.idx, self.n_sel, self.src_skv, self.skv,
+                           self.stream)
+
     def call(self, entry="attn_fwd"):
+        if entry == "gather":
+            return self.gather()
+        if self.topk and entry == "attn_fwd":
+            self.gather()
         rc = self.b.fwd_raw(*self.args(), entry=entry)
         if rc != 0:
             raise self.b.AttnError(rc, entry)
@@ -225,7 +254,7 @@ class GpuRunner:
         return self.plan["path"] == 1
 
     def launches_per_step(self):
-        return 2 if self.decode else 1
+        return (2 if self.decode else 1) + (1 if self.topk else 0)
 
     def _graph(self, nsteps, entry="attn_fwd"):
         """Capture `nsteps` launches of `entry` (a whole step for attn_fwd)
@@ -262,7 +291,8 @@ class GpuRunner:
         The dominant kernel's duration is timed the same way over graphs of
         20 back-to-back launches of that kernel alone (for decode the split
         kernel, whose inputs do not depend on the combine); the combine's is
-        the step time minus that."""
+        the step time minus that (and minus the row gather of a top-k step,
+        timed the same way, in ``self.gather_ms``)."""
         per = max(d for d in range(1, min(steps, 20) + 1) if steps % d == 0)
         graph, side = self._graph(per)
         total = self._replay_ms(graph, side, steps // per, max(1, warmup // per))
@@ -271,29 +301,44 @@ class GpuRunner:
             return total, total / steps, 0.0
         kg, kside = self._graph(20, "attn_decode_partial")
         k_ms = self._replay_ms(kg, kside, 10, 1) / 200
-        return total, k_ms, max(total / steps - k_ms, 0.0)
+        del kg
+        self.gather_ms = 0.0
+        if self.topk:
+            gg, gside = self._graph(20, "gather")
+            self.gather_ms = self._replay_ms(gg, gside, 10, 1) / 200
+            del gg
+        return total, k_ms, max(total / steps - k_ms - self.gather_ms, 0.0)
 
     def e2e(self, steps, warmup, inp):
         """Same step through the C ABI with the step's inputs in pinned host
         memory: H2D copy of the inputs, the forward, D2H copy of out and lse,
         synchronised every step.  Decode keeps the KV cache resident (it is
-        state, not a per-step input); prefill copies q, k and v every step."""
+        state, not a per-step input); prefill copies q, k and v every step;
+        a top-k step also copies the selection (idx, n_sel)."""
         pin = lambda t: t.pin_memory()
         hq = pin(inp["q"])
         hskv = pin(inp["skv"])
-        hk = hv = None
+        hk = hv = hidx = hnsel = None
+        dskv = self.src_skv if self.topk else self.skv
         if not self.decode:  # prefill shapes have separate K and V tensors
             hk, hv = pin(inp["k"]), pin(inp["v"])
+        if self.topk:
+            hidx, hnsel = pin(inp["idx"]), pin(inp["n_sel"])
         hout = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         hlse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
         h2d = hq.numel() * hq.element_size() + hskv.numel() * 4
         if hk is not None:
             h2d += hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+        if hidx is not None:
+            h2d += hidx.numel() * 4 + hnsel.numel() * 4
         d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
 
         def step():
             self.q.copy_(hq, non_blocking=True)
-            self.skv.copy_(hskv, non_blocking=True)
+            dskv.copy_(hskv, non_blocking=True)
+            if hidx is not None:
+                self.idx.copy_(hidx, non_blocking=True)
+                self.n_sel.copy_(hnsel, non_blocking=True)
             if hk is not None:
                 self.k.copy_(hk, non_blocking=True)
                 self.v.copy_(hv, non_blocking=True)
@@ -349,7 +394,14 @@ def config_of(w, inp, parallelism):
          "d_v": w.d_v, "causal": w.causal, "scale": round(w.scale, 6), "mla_absorbed": w.mla,
          "skv": f"U[{w.skv_lo},{w.skv_hi}] seed {w.seed}" if w.skv_lo != w.skv_hi else w.skv_lo,
          "skv_total": int(skv.sum()), "parallelism": parallelism}
-    if w.is_decode:
+    if w.topk:
+        sel = kv_bytes(w, inp["n_sel"])
+        d["topk"] = w.topk
+        d["selection"] = ("per sequence min(topk, skv) distinct positions, uniform, ascending "
+                          f"(seed {w.seed}); {int(inp['n_sel'].sum())} rows selected")
+        d["l2"] = (f"inputs larger than L2: selected rows {sel / 1e6:.0f} MB > 126 MB, gathered "
+                   "from a {:.1f} GB cache".format(kv_bytes(w, skv) / 1e9))
+    elif w.is_decode:
         d["l2"] = f"inputs larger than L2: KV {kv_bytes(w, skv) / 1e6:.0f} MB > 126 MB"
     else:
         qb = w.B * w.Hq * w.Sq * w.d_k * 2
@@ -362,7 +414,11 @@ def config_of(w, inp, parallelism):
 
 def oracle_sample(w, inp, budget_s):
     """The first n sequences (all heads) whose estimated oracle cost fits the
-    budget (the fp64 C oracle runs at roughly 1 GFLOP/s per thread)."""
+    budget (the fp64 C oracle runs at roughly 1 GFLOP/s per thread; the
+    numpy top-k oracle is timed on one sequence)."""
+    if w.topk:
+        t1 = max(run_oracle(w, inp, 1), 1e-3)
+        return max(1, min(w.B, int(budget_s / t1)))
     rate = 1.0e9 * (os.cpu_count() or 1)
     skv = inp["skv"].tolist()
     n, acc = 0, 0.0
@@ -379,13 +435,19 @@ def run_oracle(w, inp, n):
     from oracle import c_oracle
 
     t0 = time.perf_counter()
-    c_oracle.attention_fwd(inp["q"][:n], inp["k"][:n], inp["v"][:n], inp["skv"][:n].tolist(),
-                           w.scale, w.causal)
+    if w.topk:
+        from oracle import attention as npo
+
+        npo.topk_attention_fwd(inp["q"][:n], inp["k"][:n], inp["v"][:n], inp["skv"][:n].tolist(),
+                               inp["idx"][:n], inp["n_sel"][:n].tolist(), w.scale)
+    else:
+        c_oracle.attention_fwd(inp["q"][:n], inp["k"][:n], inp["v"][:n],
+                               inp["skv"][:n].tolist(), w.scale, w.causal)
     return time.perf_counter() - t0
 
 
 def cpu_value(w, inp, n, secs):
-    skv = inp["skv"][:n].tolist()
+    skv = keys_of(w, inp)[:n].tolist()
     wb = w.scaled(B=n)
     if w.is_decode:
         return kv_bytes(wb, skv) / secs / 1e9
@@ -446,7 +508,8 @@ def reference_arm(args, world, rank):
     val = cpu_value(w, inp, n, t / steps)
     metric, unit, hib = metric_of(w)
     cores = os.cpu_count() or 1
-    sample = f"first {n} of {w.B} sequences, all {w.Hq} heads, per step"
+    sample = f"first {n} of {w.B} sequences, all {w.Hq} heads, per step" + (
+        " (numpy fp64 top-k oracle)" if w.topk else "")
     line = {"impl": "reference", "metric": f"{w.name}_{metric}", "value": round(val, 4),
             "unit": unit, "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": round(t / steps * 1e3, 3), "higher_is_better": hib,
@@ -515,7 +578,8 @@ def main():
     import torch.distributed as dist_mod
 
     max_ms = allreduce(total_ms, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
-    work = kv_bytes(w, inp["skv"]) if w.is_decode else flops(w, inp["skv"])
+    keys = keys_of(w, inp)
+    work = kv_bytes(w, keys) if w.is_decode else flops(w, keys)
     work_all = allreduce(work, dist_mod.ReduceOp.SUM if world > 1 else None, world, device)
     ms_step = max_ms / steps
     scale_div = 1e9 if w.is_decode else 1e12
@@ -523,11 +587,17 @@ def main():
     metric, unit, hib = metric_of(w)
     long_run = total_ms > 1000.0
     kname = ("mla_pair_kernel" if w.mla else "decode_split_kernel") if g.decode else "prefill_kernel"
-    roof = roofline(w, inp["skv"], k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
+    roof = roofline(w, keys, k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
     roof["kernel"] = kname
     roof["kernel_ms"] = round(k_ms, 5)
     if g.decode:
         roof["combine_ms"] = round(other_ms, 5)
+    if w.topk:  # the row gather: reads and writes the selected rows once each
+        gb = 2 * kv_bytes(w, keys) / (g.gather_ms * 1e-3) / 1e9
+        roof["gather"] = {"kernel": "gather_rows_kernel", "ms": round(g.gather_ms, 5),
+                          "bytes_per_launch": 2 * kv_bytes(w, keys), "achieved": round(gb, 1),
+                          "frac": round(gb / float(peaks["hbm_gbs"]), 4), "unit": "GB/s",
+                          "traffic": traffic_for("gather_rows_kernel", w.name)}
 
     # end to end through the C ABI with host buffers
     e2e_steps = max(10, min(steps, 200))
@@ -575,10 +645,11 @@ def main():
 
         c_oracle.build()
         secs = run_oracle(w, inp, n)
+        which = "numpy fp64 top-k oracle" if w.topk else "fp64 C oracle"
         line["cpu_baseline"] = {"value": round(cpu_value(w, inp, n, secs), 4), "unit": unit,
                                 "cores": os.cpu_count() or 1, "kind": "oracle",
                                 "sample": f"first {n} of {w.B} sequences, all {w.Hq} heads "
-                                          f"({secs:.1f} s, fp64 C oracle)"}
+                                          f"({secs:.1f} s, {which})"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

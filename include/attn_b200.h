@@ -65,7 +65,8 @@ typedef enum {
   ATTN_EWORKSPACE = 3,    /* workspace missing or smaller than required        */
   ATTN_ECUDA = 4,         /* a CUDA runtime/driver call or launch failed       */
   ATTN_ETIMEOUT = 5,      /* a device-side wait gave up (see attn_last_device_error) */
-  ATTN_EOVERFLOW = 6      /* attn_cache_append found a full sequence (see attn_last_device_error) */
+  ATTN_EOVERFLOW = 6,     /* attn_cache_append found a full sequence (see attn_last_device_error) */
+  ATTN_EINDEX = 7         /* attn_gather_rows met a position outside its sequence (ditto) */
 } attn_status_t;
 
 typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype_t;
@@ -190,7 +191,8 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void
  * error word.  ATTN_OK if no kernel of this library reported a problem
  * since the last call, ATTN_ETIMEOUT if a device-side wait gave up (the
  * outputs of that launch are undefined), ATTN_EOVERFLOW if attn_cache_append
- * met a full sequence, ATTN_ECUDA if the stream itself reports an error.
+ * met a full sequence, ATTN_EINDEX if attn_gather_rows met a position outside
+ * its sequence, ATTN_ECUDA if the stream itself reports an error.
  */
 attn_status_t attn_last_device_error(void* cuda_stream);
 
@@ -219,6 +221,29 @@ attn_status_t attn_cache_append(void* k_cache, void* v_cache, const void* k_new,
                                 int32_t* skv_per_seq, int B, int Hkv, int max_skv, int d_k,
                                 int d_v, attn_dtype_t dtype, attn_strides_t sk, attn_strides_t sv,
                                 attn_strides_t skn, attn_strides_t svn, void* cuda_stream);
+
+/*
+ * Top-k sparse decode in the DSA style ("带你了解Attention,从MHA到DeepSeek"
+ * section 5.1: an indexer -- not part of this library -- selects the top-k
+ * cached entries for each new token; attention then runs over those only):
+ * copies, for every sequence b and head h < H, the rows at the selected
+ * positions idx[b * idx_stride + t], t < n_sel[b] (at most topk), of
+ * src [B, H, >= skv[b], d] into dst [B, H, >= topk, d] in selection order,
+ * and writes dst_len[b] = n_sel[b].  An attn_fwd on (q, dst, dst_len) on the
+ * same stream is then attention over the selected keys (for MLA pass dst as
+ * both k and v with d = 576).  A position outside [0, skv[b]) yields a zero
+ * row and sets bit 2 of the device error word (ATTN_EINDEX from
+ * attn_last_device_error).
+ * - idx, n_sel, skv_per_seq, dst_len: device int32; src/dst: element
+ *   strides s_src / s_dst (innermost contiguous), 16-byte aligned, d a
+ *   multiple of 8.  Errors before launch: ATTN_EINVAL; ATTN_EUNSUPPORTED for
+ *   B or H above 65535; ATTN_ECUDA on a launch error.
+ */
+attn_status_t attn_gather_rows(const void* src, void* dst, const int32_t* idx,
+                               const int32_t* n_sel, const int32_t* skv_per_seq, int32_t* dst_len,
+                               int B, int H, int topk, int d, attn_dtype_t dtype,
+                               attn_strides_t s_src, attn_strides_t s_dst, int64_t idx_stride,
+                               void* cuda_stream);
 
 /* Bound on every device-side wait of launches made after this call, in
  * nanoseconds of %globaltimer (process-wide; 0 restores the default of 2 s).

@@ -192,7 +192,7 @@ def topk_attention_fwd(q, k, v, skv_lens, idx, n_sel, scale: float):
     causal mask beyond the selection).  A position listed twice counts twice.
     n_sel[b] == 0 gives out 0, lse -inf.  Positions outside [0, skv[b]) raise.
     Returns (out [B, Hq, Sq, d_v], lse [B, Hq, Sq]) in float64."""
-    q, k, v = _f64(q), _f64(k), _f64(v)
+    q = _f64(q)
     idx = np.asarray(idx.tolist() if hasattr(idx, "tolist") else idx, dtype=np.int64)
     B, Hq, Sq, _ = q.shape
     Hkv, d_v = k.shape[1], v.shape[-1]
@@ -206,8 +206,11 @@ def topk_attention_fwd(q, k, v, skv_lens, idx, n_sel, scale: float):
         sel = idx[b, :n]
         if sel.min() < 0 or sel.max() >= int(skv_lens[b]):
             raise ValueError(f"sequence {b}: a selected position lies outside [0, skv)")
+        # only the selected rows are widened to float64 (long caches stay compact)
+        ti = sel.tolist()
+        ks, vs = _f64(k[b][:, ti]), _f64(v[b][:, ti])  # [Hkv, n, d]
         for h in range(Hq):
-            kh, vh = k[b, h // G][sel], v[b, h // G][sel]  # [n, d]
+            kh, vh = ks[h // G], vs[h // G]  # [n, d]
             s = scale * (q[b, h] @ kh.T)  # [Sq, n]
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)

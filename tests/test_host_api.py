@@ -33,7 +33,7 @@ def test_header_declarations_are_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert binding.status_str(code) and binding.status_str(code) != "unknown status"
     assert binding.version().count(".") == 2
 
@@ -211,3 +211,28 @@ def test_cache_append_rejects_before_launch(lib, over, code):
     assert lib.attn_cache_append(a["kc"], a["vc"], a["kn"], a["vn"], a["skv"], a["B"], a["Hkv"],
                                  a["max_skv"], a["dk"], a["dv"], a["dtype"], s, s, sn, sn,
                                  None) == code
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(src=None), binding.ATTN_EINVAL),
+    (dict(idx=None), binding.ATTN_EINVAL),
+    (dict(dst_len=None), binding.ATTN_EINVAL),
+    (dict(idx=0x50002), binding.ATTN_EINVAL),            # int32 array not 4-byte aligned
+    (dict(dst=0x20008), binding.ATTN_EINVAL),            # not 16-byte aligned
+    (dict(d=100), binding.ATTN_EINVAL),                  # not a multiple of 8 elements
+    (dict(topk=0), binding.ATTN_EINVAL),
+    (dict(idx_stride=8), binding.ATTN_EINVAL),           # rows shorter than topk
+    (dict(dtype=5), binding.ATTN_EINVAL),
+    (dict(H=70000), binding.ATTN_EUNSUPPORTED),
+])
+def test_gather_rows_rejects_before_launch(lib, over, code):
+    """attn_gather_rows validates its arguments before anything reaches the
+    device (the fake pointers below are never dereferenced)."""
+    a = dict(src=0x10000, dst=0x20000, idx=0x50000, n_sel=0x60000, skv=0x70000,
+             dst_len=0x80000, B=2, H=1, topk=16, d=576, dtype=0, idx_stride=16)
+    a.update(over)
+    ss = binding.Strides(4096 * a["d"], 4096 * a["d"], a["d"])
+    sd = binding.Strides(16 * a["d"], 16 * a["d"], a["d"])
+    assert lib.attn_gather_rows(a["src"], a["dst"], a["idx"], a["n_sel"], a["skv"], a["dst_len"],
+                                a["B"], a["H"], a["topk"], a["d"], a["dtype"], ss, sd,
+                                a["idx_stride"], None) == code
