@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -224,11 +225,25 @@ enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
 // only before reading the partials, so its launch and prologue overlap the
 // split kernel's tail.
 template <bool BF16>
-attn_status_t launch_combine(const attn::DecodeParams& dp, const attn::CombineParams& cp,
+attn_status_t launch_combine(const attn::DecodeParams& dp, attn::CombineParams cp,
                              cudaStream_t st) {
+  (void)dp;
+  // Columns per block: as many as keep a block's outputs within 1024 float4
+  // (8 per thread), then halved while the grid would leave SMs idle (down to
+  // one float4 per thread).
+  const int GC = cp.G * cp.Sq;
+  const int D4 = cp.DV / 4;
+  const long long units = (long long)cp.B * cp.Hkv;
+  int cc = 1;
+  while (cc * 2 <= GC && cc * 2 * D4 <= 1024 && cc * 2 <= 32) cc *= 2;
+  const long long target = 2LL * device_sm_count();
+  while (cc > 1 && cc * D4 > attn::kCombineThreads && units * ((GC + cc - 1) / cc) < target) cc /= 2;
+  cp.cols = cc;
+  cp.col_chunks = (GC + cc - 1) / cc;
+  const int fpt = std::max(1, cc * D4 / attn::kCombineThreads);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(dp.B * dp.Hq * dp.Sq), 1, 1);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.gridDim = dim3((unsigned)(units * cp.col_chunks), 1, 1);
+  cfg.blockDim = dim3(attn::kCombineThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -236,7 +251,14 @@ attn_status_t launch_combine(const attn::DecodeParams& dp, const attn::CombinePa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16>, cp) != cudaSuccess) {
+  cudaError_t e;
+  switch (fpt) {
+    case 1: e = cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16, 1>, cp); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16, 2>, cp); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16, 4>, cp); break;
+    default: e = cudaLaunchKernelEx(&cfg, attn::combine_kernel<BF16, 8>, cp); break;
+  }
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ECUDA;
   }

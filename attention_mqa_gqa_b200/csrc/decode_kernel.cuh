@@ -702,153 +702,6 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
   }
 }
 
-// ---------------------------------------------------------------- combine
-//
-// out[b,h,i,:] = sum_s exp(lse_s - L) o_s,  L = log sum_s exp(lse_s), over
-// the pieces of unit (b, h / G), in range order (no atomics, so the result
-// is bitwise reproducible: "GQA和MLA详解" section 4 on reduction order).
-struct CombineParams {
-  const float* ws_o;
-  const float* ws_lse;
-  const int32_t* skv;
-  void* out;
-  int64_t o_sb, o_sh;
-  int64_t o_ss;
-  float* lse;  // [B, Hq, Sq] or NULL
-  int B, Hq, Hkv, G, DV, ranges;
-  int Sq;          // queries per sequence (columns per head)
-  int tile_shift;  // log2 of the keys per tile the partial kernel used
-};
-
-// Largest range index r with floor(r * T / R) <= x (the range holding tile x).
-__device__ __forceinline__ long long range_of(long long x, long long T, long long R) {
-  return ((x + 1) * R + T - 1) / T - 1;
-}
-
-template <bool BF16>
-__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
-  // One block per (b, h, query i).  The piece weights w_s = exp(lse_s - L) are
-  // computed once into shared memory; each thread then owns 4 consecutive
-  // d_v columns (float4) of one piece-group g and accumulates its pieces
-  // s = g, g + NG, ... in order; the NG group sums are added in group order.
-  constexpr int MAXS = 1024;
-  __shared__ float w_sm[MAXS];
-  __shared__ float red[4];
-  __shared__ long long redl[8];
-  __shared__ float4 part[128];
-  const int bhi = blockIdx.x;  // (b, h, query i)
-  const int qi = bhi % p.Sq;
-  const int bh = bhi / p.Sq;
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
-  const int kvh = h / p.G;
-  const int gh = (h % p.G) * p.Sq + qi;  // column within the kv head's G * Sq
-  const int GC = p.G * p.Sq;
-  const int t = threadIdx.x;
-  const int warp = t >> 5, lane = t & 31;
-
-  // tiles of the sequences before b, and of all sequences
-  long long pre = 0, tot = 0;
-  for (int bb = t; bb < p.B; bb += 128) {
-    const int tb = key_tiles(p.skv[bb], p.tile_shift);
-    tot += tb;
-    if (bb < b) pre += tb;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    pre += __shfl_xor_sync(0xffffffffu, pre, o);
-    tot += __shfl_xor_sync(0xffffffffu, tot, o);
-  }
-  if (lane == 0) {
-    redl[warp] = pre;
-    redl[4 + warp] = tot;
-  }
-  __syncthreads();
-  pre = (redl[0] + redl[1]) + (redl[2] + redl[3]);
-  tot = (redl[4] + redl[5]) + (redl[6] + redl[7]);
-  const int tu = key_tiles(p.skv[b], p.tile_shift);
-  const long long T = tot * p.Hkv;
-  // Everything above reads inputs only; the partials come from the kernel
-  // before this one in the stream, which may still be running.
-  pdl_wait();
-  const long long Re = T < p.ranges ? T : p.ranges;  // ranges in use, none empty
-  const long long u = (long long)b * p.Hkv + kvh;
-  int n = 0;
-  long long r_lo = 0;
-  if (tu > 0) {
-    const long long su = pre * p.Hkv + (long long)kvh * tu;
-    r_lo = range_of(su, T, Re);
-    n = (int)(range_of(su + tu - 1, T, Re) - r_lo + 1);
-    n = min(n, MAXS);
-  }
-  // piece s of this unit lives in workspace slot (r_lo + s) + u
-  auto slot = [&](int s) { return (r_lo + s + u) * GC + gh; };
-
-  float mx = -INFINITY;
-  for (int s = t; s < n; s += 128) mx = fmaxf(mx, p.ws_lse[slot(s)]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  float sum = 0.f;
-  if (mx != -INFINITY)
-    for (int s = t; s < n; s += 128) sum += __expf(p.ws_lse[slot(s)] - mx);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) red[warp] = sum;
-  __syncthreads();
-  sum = (red[0] + red[1]) + (red[2] + red[3]);
-  const float L = (mx == -INFINITY || !(sum > 0.f)) ? -INFINITY : mx + __logf(sum);
-  for (int s = t; s < n; s += 128) w_sm[s] = (L == -INFINITY) ? 0.f : __expf(p.ws_lse[slot(s)] - L);
-  __syncthreads();
-
-  const int D4 = p.DV / 4;             // float4 columns (128 or 32)
-  const int NG = 128 / D4;             // piece groups (1 or 4)
-  const int d4 = t % D4;
-  const int g = t / D4;
-  auto src = [&](int s) {
-    return reinterpret_cast<const float4*>(p.ws_o + slot(s) * (long long)p.DV)[d4];
-  };
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = g;
-  for (; s + 3 * NG < n; s += 4 * NG) {  // four independent loads in flight
-    const float4 v0 = src(s), v1 = src(s + NG), v2 = src(s + 2 * NG), v3 = src(s + 3 * NG);
-    const float w0 = w_sm[s], w1 = w_sm[s + NG], w2 = w_sm[s + 2 * NG], w3 = w_sm[s + 3 * NG];
-    acc.x = fmaf(w3, v3.x, fmaf(w2, v2.x, fmaf(w1, v1.x, fmaf(w0, v0.x, acc.x))));
-    acc.y = fmaf(w3, v3.y, fmaf(w2, v2.y, fmaf(w1, v1.y, fmaf(w0, v0.y, acc.y))));
-    acc.z = fmaf(w3, v3.z, fmaf(w2, v2.z, fmaf(w1, v1.z, fmaf(w0, v0.z, acc.z))));
-    acc.w = fmaf(w3, v3.w, fmaf(w2, v2.w, fmaf(w1, v1.w, fmaf(w0, v0.w, acc.w))));
-  }
-  for (; s < n; s += NG) {
-    const float4 v = src(s);
-    const float wv = w_sm[s];
-    acc.x = fmaf(wv, v.x, acc.x);
-    acc.y = fmaf(wv, v.y, acc.y);
-    acc.z = fmaf(wv, v.z, acc.z);
-    acc.w = fmaf(wv, v.w, acc.w);
-  }
-  if (NG > 1) {
-    part[t] = acc;
-    __syncthreads();
-    if (g == 0) {
-      for (int gg = 1; gg < NG; ++gg) {
-        const float4 o = part[gg * D4 + d4];
-        acc.x += o.x;
-        acc.y += o.y;
-        acc.z += o.z;
-        acc.w += o.w;
-      }
-    }
-  }
-  if (g == 0) {
-    uint8_t* outp =
-        reinterpret_cast<uint8_t*>(p.out) +
-        ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)qi * p.o_ss + d4 * 4) * 2;
-    *reinterpret_cast<uint2*>(outp) = make_uint2(pack2(acc.x, acc.y, BF16), pack2(acc.z, acc.w, BF16));
-  }
-  if (t == 0 && p.lse) p.lse[bhi] = L;
-}
-
 }  // namespace attn
+
+#include "combine_kernel.cuh"
