@@ -100,11 +100,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_tokens(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace runs collapsed
+    (string and character literals kept verbatim): what the compiler sees,
+    so that editing a comment does not void a recorded measurement."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == "/" and text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif c == "/" and text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def sources_hash(kernel: str) -> str:
+    """Hash of the code (comments and layout ignored) a kernel is built from."""
     h = hashlib.sha256()
     for s in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, s), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, s), encoding="utf-8") as f:
+            h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,0 +1,54 @@
+"""Host-side pieces of bench.py and the input generators (no GPU): the
+source fingerprint that gates recorded DRAM traffic, the top-k accounting,
+and the top-k selection generator."""
+import json
+import os
+
+import torch
+
+import bench
+from attention_mqa_gqa_b200 import workloads as wl
+
+
+def test_code_tokens_drops_comments_keeps_literals():
+    src = ('int a = 1; // note\n/* block\n comment */ const char* s = "x // y /* z */";\n'
+           "char q = '\"';   int   b;  // it's\n")
+    assert bench.code_tokens(src) == 'int a = 1; const char* s = "x // y /* z */"; char q = \'"\'; int b;'
+    # re-wrapping or rewording a comment leaves the fingerprint unchanged; code does not
+    assert bench.code_tokens("x = 1; // one\n") == bench.code_tokens("x  =  1;\n// two\n")
+    assert bench.code_tokens("x = 1;") != bench.code_tokens("x = 2;")
+
+
+def test_recorded_traffic_matches_current_sources():
+    """Every committed ncu traffic figure was taken on the kernel code as it
+    is now (else bench.py reports traffic null)."""
+    with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
+        d = json.load(f)
+    for key, e in d.items():
+        kernel, workload = key.split(":")
+        assert e["sources_sha"] == bench.sources_hash(kernel), key
+        assert bench.traffic_for(kernel, workload) == e["dram_bytes_per_launch"]
+
+
+def test_make_selection():
+    g = torch.Generator().manual_seed(0)
+    skv = [5000, 100, 0, 2048]
+    idx, n_sel = wl.make_selection(skv, 2048, g)
+    assert n_sel.tolist() == [2048, 100, 0, 2048]
+    for b, L in enumerate(skv):
+        sel = idx[b, : n_sel[b]]
+        assert len(set(sel.tolist())) == len(sel)              # distinct
+        assert bool((sel[1:] > sel[:-1]).all())                 # ascending
+        assert len(sel) == 0 or (0 <= int(sel.min()) and int(sel.max()) < L)
+    assert sorted(idx[3].tolist()) == list(range(2048))         # skv == topk: every position
+
+
+def test_topk_accounting():
+    """A top-k step reads the selected rows once: kv bytes = selected rows x
+    1152 B for the 576-wide latent rows."""
+    w = wl.WORKLOADS["mla_topk_decode"].scaled(B=3, skv_lo=100, skv_hi=3000)
+    inp = {"skv": torch.tensor([3000, 100, 2500], dtype=torch.int32),
+           "n_sel": torch.tensor([2048, 100, 2048], dtype=torch.int32)}
+    assert w.is_decode
+    assert bench.keys_of(w, inp).tolist() == [2048, 100, 2048]
+    assert bench.kv_bytes(w, bench.keys_of(w, inp)) == (2048 + 100 + 2048) * 576 * 2
