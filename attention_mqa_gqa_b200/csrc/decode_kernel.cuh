@@ -1,32 +1,37 @@
-// decode_kernel.cuh -- persistent split-KV decode (one query row per head,
-// Sq == 1) and the LSE combine.
+// decode_kernel.cuh -- persistent split-KV decode: one query per head
+// (Sq == 1), or a few (Sq = 2..16, a power of two: extend / speculative
+// verification) against the KV cache, head dim 128 or 512.
 //
 // Decode reads the whole KV cache once per step and is bandwidth-bound
 // ("GQA和MLA详解" section 1; "Full 路线" section 4.5), so every K/V byte
 // must be read from HBM once for all G query heads that share it
 // ("GQA和MLA详解" section 2: real kernels index the shared head instead of
 // copying it).  This kernel puts 128 keys of one KV head in the MMA M
-// dimension and the group's query heads in N:
+// dimension and NH = 16 columns in N, a column being one (query head,
+// query) pair of the group:
 //
-//   S^T[128 keys x NH heads] = K_tile[128 x d_k] * Q^T          (tcgen05, TMEM)
-//   softmax over keys per head (online, with a lazily raised max)
-//   O^T[d_v x NH]           += V_tile^T[d_v x 128] * P^T[128 x NH]
+//   S^T[128 keys x NH] = K_tile[128 x d_k] * Q^T                 (tcgen05, TMEM)
+//   softmax over keys per column (online, with a lazily raised max)
+//   O^T[d_v x NH]     += V_tile^T[d_v x 128] * P^T[128 x NH]
 //
-// so 16 MQA heads, 8 GQA heads (padded to 16) and 64 of the 128 MLA heads
-// use the tensor cores without padding M with absent query rows.
+// so the 16 heads of MQA, or the 8 heads of a GQA group (N padded to 16, or
+// filled by 8 heads x 2 queries), use the tensor cores without padding the
+// 128-row M dimension with absent query rows.  With Sq > 1 each column
+// carries its own bottom-right causal limit.
 //
 // Scheduling: the grid is persistent (one wave).  The key tiles of all
 // (sequence, kv head) units, laid end to end, are cut into `ranges` equal
 // contiguous ranges; each CTA (with one CTA per head block of the group)
 // walks its range, which may span several units.  Each maximal piece of a
 // unit inside a range produces one normalised partial output and its LSE
-// in slot (range + unit) of the workspace; the combine kernel merges the
+// in slot (range + unit) of the workspace; combine_kernel.cuh merges the
 // pieces of each unit in range order.  Every SM gets the same number of
-// key tiles whatever the mix of sequence lengths.
+// key tiles whatever the mix of sequence lengths.  A sequence's partial
+// last tile is read as the 128 rows ending at its last key, so no cache row
+// past the sequence is ever read.
 //
-// MLA absorbed mode ("Full 路线" sections 4.2-4.3): K rows are the cached
-// [c_kv | k_pe] rows (d_k = 576) and V is the first 512 columns of the same
-// rows (d_v = 512), read through a second tensor map over the same memory.
+// The absorbed-MLA rows (d_k = 576, V = their first 512 columns) run on
+// SM pairs in mla_pair_kernel.cuh, which reuses the scheduling here.
 //
 // Warp roles (320 threads): warp 0 lane 0 streams K/V chunks through the
 // ring and lane 1 loads Q^T per piece (both TMA), warp 1 allocates TMEM and
