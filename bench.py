@@ -299,18 +299,26 @@ class GpuRunner:
         self.stream, self._args = saved, None
         return graph, side
 
-    def _replay_ms(self, graph, side, reps, warmup_reps):
+    def _replay_ms(self, graph, side, reps, warmup_reps, per_replay=None):
+        """Total ms of `reps` back-to-back replays (events on the replay
+        stream); with a list in `per_replay`, also each replay's ms (an event
+        between consecutive replays, so the replays still run back to back)."""
         with torch.cuda.stream(side):  # replays run on the current stream
             for _ in range(warmup_reps):
                 graph.replay()
             torch.cuda.synchronize(self.dev)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(side)
-            for _ in range(reps):
+            ev = [torch.cuda.Event(enable_timing=True)
+                  for _ in range(reps + 1 if per_replay is not None else 2)]
+            ev[0].record(side)
+            for r in range(reps):
                 graph.replay()
-            b.record(side)
+                if per_replay is not None:
+                    ev[r + 1].record(side)
+            ev[-1].record(side)
             torch.cuda.synchronize(self.dev)
-        return a.elapsed_time(b)
+        if per_replay is not None:
+            per_replay.extend(ev[r].elapsed_time(ev[r + 1]) for r in range(reps))
+        return ev[0].elapsed_time(ev[-1])
 
     def timed(self, steps, warmup):
         """Warm up, then time exactly `steps` steps replayed from CUDA graphs
@@ -323,7 +331,9 @@ class GpuRunner:
         timed the same way, in ``self.gather_ms``)."""
         per = max(d for d in range(1, min(steps, 20) + 1) if steps % d == 0)
         graph, side = self._graph(per)
-        total = self._replay_ms(graph, side, steps // per, max(1, warmup // per))
+        reps = []
+        total = self._replay_ms(graph, side, steps // per, max(1, warmup // per), reps)
+        self.step_ms_samples = [r / per for r in reps]  # mean step time of each replay
         del graph
         if not self.decode:
             return total, total / steps, 0.0
@@ -459,7 +469,9 @@ def oracle_sample(w, inp, budget_s):
     return n
 
 
-def run_oracle(w, inp, n):
+def run_oracle(w, inp, n, nthreads=None):
+    """Seconds the oracle takes on the first n sequences (all heads); the C
+    oracle on `nthreads` host threads (default: all cores)."""
     from oracle import c_oracle
 
     t0 = time.perf_counter()
@@ -470,7 +482,7 @@ def run_oracle(w, inp, n):
                                inp["idx"][:n], inp["n_sel"][:n].tolist(), w.scale)
     else:
         c_oracle.attention_fwd(inp["q"][:n], inp["k"][:n], inp["v"][:n],
-                               inp["skv"][:n].tolist(), w.scale, w.causal)
+                               inp["skv"][:n].tolist(), w.scale, w.causal, nthreads=nthreads)
     return time.perf_counter() - t0
 
 
@@ -615,6 +627,10 @@ def main():
     metric, unit, hib = metric_of(w)
     long_run = total_ms > 1000.0
     kname = ("mla_pair_kernel" if w.mla else "decode_split_kernel") if g.decode else "prefill_kernel"
+    samples = sorted(g.step_ms_samples)
+    pct = lambda q: samples[min(len(samples) - 1, int(q * (len(samples) - 1) + 0.5))]
+    step_dist = {"p10": round(pct(0.1), 5), "p50": round(pct(0.5), 5), "p90": round(pct(0.9), 5),
+                 "replays": len(samples), "steps_per_replay": steps // len(samples)}
     roof = roofline(w, keys, k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
     roof["kernel"] = kname
     roof["kernel_ms"] = round(k_ms, 5)
@@ -636,7 +652,8 @@ def main():
 
     line = {"metric": f"{w.name}_{metric}", "value": round(value, 3), "unit": unit,
             "n_gpus": world, "steps": steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_step, 5), "higher_is_better": hib, "scaling": "weak",
+            "ms_per_step": round(ms_step, 5), "ms_per_step_dist": step_dist,
+            "higher_is_better": hib, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "fp16",
             "data": "synthetic (seeded N(0,1), rounded once to the element type)",
             "config": config_of(w, inp, f"replicas x{world}" if world > 1 else "single GPU"),
@@ -678,6 +695,11 @@ def main():
                                 "cores": os.cpu_count() or 1, "kind": "oracle",
                                 "sample": f"first {n} of {w.B} sequences, all {w.Hq} heads "
                                           f"({secs:.1f} s, {which})"}
+        if not w.topk:  # the same oracle on one host thread, first sequence
+            s1 = run_oracle(w, inp, 1, nthreads=1)
+            line["cpu_baseline"]["value_1core"] = round(cpu_value(w, inp, 1, s1), 4)
+            line["cpu_baseline"]["sample_1core"] = (f"first sequence, all {w.Hq} heads, one thread "
+                                                    f"({s1:.2f} s)")
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Small cases compare every output element; the full-size workloads compare
-sampled rows (the oracle evaluates those rows one by one).  Tolerance:
+Small cases and the full-size decode workloads compare every output
+element; the full-size prefill workloads compare sampled rows (the oracle
+evaluates those rows one by one).  Tolerance:
 |gpu - oracle| <= 1e-2 + 1e-2*|oracle| per element, |dLSE| <= 1e-3.
 """
 import math
@@ -207,7 +208,7 @@ def test_bitwise_reproducible():
 
 # ------------------------------------------------------- full-size workloads
 
-def _sampled(name, n_pairs=12, n_rows=48, seed=0):
+def _sampled(name, n_rows=48, seed=0):
     from oracle import attention as npo
     from oracle import c_oracle
 
@@ -216,12 +217,11 @@ def _sampled(name, n_pairs=12, n_rows=48, seed=0):
     out, lse = run_gpu(w, to_device(inp))
     rng = np.random.default_rng(seed)
     if w.is_decode:
-        pairs = [(int(rng.integers(w.B)), int(rng.integers(w.Hq))) for _ in range(n_pairs)]
-        pairs += [(0, 0), (w.B - 1, w.Hq - 1)]
+        # decode reads each cached row once per head group: the fp64 oracle
+        # covers every output element of the batch in seconds (all host threads)
         ref_o, ref_l = c_oracle.attention_fwd(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(),
-                                              w.scale, w.causal, pairs=pairs)
-        for (b, h) in pairs:
-            compare(out[b, h], lse[b, h], ref_o[b, h], ref_l[b, h], f"{name} b={b} h={h}")
+                                              w.scale, w.causal)
+        compare(out, lse, ref_o, ref_l, f"{name} (every element)")
     else:
         rows = [(int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.Sq)))
                 for _ in range(n_rows)]

@@ -3,10 +3,9 @@ at caller-selected positions are gathered (attn_gather_rows) and attention
 runs over them (attn_fwd); compared with the oracle's attention over the
 selected subset.  Also: the gathered rows are bitwise copies, ragged and
 empty selections, a position outside its sequence reported as ATTN_EINDEX,
-and sampled rows of the full-size 2048-of-16K..48K MLA workload."""
+and every output of the full-size 2048-of-16K..48K MLA workload."""
 import math
 
-import numpy as np
 import pytest
 import torch
 
@@ -99,9 +98,9 @@ def test_topk_position_outside_sequence_reports_eindex():
     assert dlen.tolist() == [4, 3]
 
 
-def test_full_workload_sampled():
-    """mla_topk_decode (B=64, 128 heads, 2048 of 16K-48K positions): four
-    whole sequences against the oracle."""
+def test_full_workload():
+    """mla_topk_decode (B=64, 128 heads, 2048 of 16K-48K positions): every
+    output element against the oracle."""
     from attention_mqa_gqa_b200 import binding
     from oracle import attention as npo
 
@@ -112,10 +111,6 @@ def test_full_workload_sampled():
                                       inp["n_sel"].cuda(), dev["skv"], w.scale, d_v=w.d_v)
     torch.cuda.synchronize()
     assert binding.last_device_error() == binding.ATTN_OK
-    rng = np.random.default_rng(3)
-    for b in sorted({0, w.B - 1, *map(int, rng.integers(w.B, size=2))}):
-        sl = slice(b, b + 1)
-        ref_o, ref_l = npo.topk_attention_fwd(inp["q"][sl], inp["k"][sl], inp["v"][sl],
-                                              inp["skv"][sl].tolist(), inp["idx"][sl],
-                                              inp["n_sel"][sl].tolist(), w.scale)
-        compare(out[sl], lse[sl], ref_o, ref_l, f"mla_topk_decode b={b}")
+    ref_o, ref_l = npo.topk_attention_fwd(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(),
+                                          inp["idx"], inp["n_sel"].tolist(), w.scale)
+    compare(out, lse, ref_o, ref_l, "mla_topk_decode (every element)")
