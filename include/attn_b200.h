@@ -30,8 +30,10 @@
  * - q: [B, Hq, Sq, d_k]; k: [B, Hkv, >= max_skv, d_k]; v: [B, Hkv,
  *   >= max_skv, d_v]; out: [B, Hq, Sq, d_v] (same element type as q);
  *   lse: [B, Hq, Sq] fp32, contiguous, may be NULL.
- * - Key rows at or past skv[b] (up to max_skv) are never weighted but are
- *   read by whole 128-row tiles; they must hold finite numbers.
+ * - Key rows at or past skv[b] (up to max_skv) are never read: they may
+ *   hold anything, e.g. memory not yet written by a growing cache (a
+ *   sequence's partial last tile is fetched as the tile-sized window that
+ *   ends at its last key).
  * - Ownership: the caller owns every buffer (q, k, v, out, lse, skv,
  *   workspace).  The library allocates no device memory and never
  *   synchronises the stream inside attn_fwd; all work is enqueued on
