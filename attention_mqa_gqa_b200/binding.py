@@ -120,6 +120,17 @@ def workspace_bytes(B, Hq, Hkv, Sq, max_skv, d_k, d_v) -> int:
     return int(load().attn_workspace_bytes(B, Hq, Hkv, Sq, max_skv, d_k, d_v))
 
 
+def _on_one_gpu(*tensors) -> None:
+    """Every tensor handed to the library is CUDA memory of one device (a
+    host pointer reaching a kernel would be an illegal access)."""
+    ts = [t for t in tensors if t is not None]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+    if len({t.device for t in ts}) > 1:
+        raise ValueError("all tensors must be on the same CUDA device")
+
+
 def _strides4(t: torch.Tensor) -> Strides:
     if t.dim() != 4 or t.stride(-1) != 1:
         raise ValueError("expected a [B, H, S, d] tensor with a contiguous last dimension")
@@ -153,6 +164,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
         raise TypeError("skv must be int32")
     if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
         raise TypeError("lse must be a contiguous float32 tensor")
+    _on_one_gpu(q, k, v, out, skv, lse, workspace)
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -178,6 +190,7 @@ def attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: tor
         raise TypeError("skv must be int32")
     if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
         raise TypeError("lse must be a contiguous float32 tensor")
+    _on_one_gpu(q, k, v, out, skv, lse)
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
     rc = load().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq,
@@ -203,6 +216,7 @@ def cache_append(k_cache: torch.Tensor, v_cache: torch.Tensor | None, k_new: tor
     B, Hkv, max_skv, d_k = k_cache.shape
     if skv.dtype != torch.int32:
         raise TypeError("skv must be int32")
+    _on_one_gpu(k_cache, v_cache, k_new, v_new, skv)
     latent = v_cache is None or v_cache.data_ptr() == k_cache.data_ptr()
     d_v = 0 if latent else v_cache.shape[-1]
     st = stream if stream is not None else torch.cuda.current_stream(k_cache.device)
@@ -233,6 +247,7 @@ def gather_rows(src: torch.Tensor, dst: torch.Tensor, idx: torch.Tensor, n_sel: 
         raise ValueError("idx rows and n_sel/skv/dst_len must be contiguous")
     if src.dtype != dst.dtype:
         raise TypeError("src and dst must have the same element type")
+    _on_one_gpu(src, dst, idx, n_sel, skv, dst_len)
     st = stream if stream is not None else torch.cuda.current_stream(dst.device)
     rc = load().attn_gather_rows(src.data_ptr(), dst.data_ptr(), idx.data_ptr(), n_sel.data_ptr(),
                                  skv.data_ptr(), dst_len.data_ptr(), B, H, topk, d,
@@ -269,8 +284,9 @@ def topk_attention(q, k_cache, v_cache, idx, n_sel, skv, scale, d_v=None, with_l
     attends over them, both on one stream.  k_cache/v_cache [B, Hkv, S, d];
     for an absorbed-MLA latent cache pass v_cache=None and d_v (the value
     rows are the first d_v columns of the gathered rows).  ``scratch`` is an
-    optional dict of preallocated device tensors (keys k, v, len, ws) reused
-    between calls.  Returns (out, lse)."""
+    optional dict the scratch tensors (keys k, v, len, ws) are kept in
+    between calls; they are reallocated when the problem's shapes change.
+    Returns (out, lse)."""
     B, Hkv, _, d_k = k_cache.shape
     topk = idx.shape[1]
     latent = v_cache is None
@@ -278,7 +294,10 @@ def topk_attention(q, k_cache, v_cache, idx, n_sel, skv, scale, d_v=None, with_l
         raise ValueError("d_v is required for a latent (MLA) cache")
     d_v = d_v if latent else v_cache.shape[-1]
     sc = scratch if scratch is not None else {}
-    if "k" not in sc:
+    key = (B, Hkv, topk, d_k, d_v, latent, k_cache.dtype, k_cache.device, q.shape[1], q.shape[2])
+    if sc.get("key") != key:  # (re)allocate for this problem's shapes
+        sc.clear()
+        sc["key"] = key
         sc["k"] = torch.empty(B, Hkv, topk, d_k, dtype=k_cache.dtype, device=k_cache.device)
         sc["v"] = None if latent else torch.empty(B, Hkv, topk, d_v, dtype=k_cache.dtype,
                                                   device=k_cache.device)

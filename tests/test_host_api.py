@@ -236,3 +236,24 @@ def test_gather_rows_rejects_before_launch(lib, over, code):
     assert lib.attn_gather_rows(a["src"], a["dst"], a["idx"], a["n_sel"], a["skv"], a["dst_len"],
                                 a["B"], a["H"], a["topk"], a["d"], a["dtype"], ss, sd,
                                 a["idx_stride"], None) == code
+
+
+def test_binding_rejects_host_tensors(lib):
+    """A CPU tensor never reaches the library: its host address would be an
+    illegal access in a kernel."""
+    import torch
+
+    q = torch.zeros(1, 16, 1, 512, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 64, 512, dtype=torch.bfloat16)
+    out = torch.zeros(1, 16, 1, 512, dtype=torch.bfloat16)
+    skv = torch.tensor([64], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.attn_fwd(q, k, k, out, skv, 64, 0.04)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.attn_fwd_noalloc(q, k, k, out, skv, 64, 0.04)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.cache_append(k, None, k[:, :, :1], None, skv)
+    idx = torch.zeros(1, 8, dtype=torch.int32)
+    dst = torch.zeros(1, 1, 8, 512, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.gather_rows(k, dst, idx, skv, skv, torch.zeros(1, dtype=torch.int32))
