@@ -13,19 +13,22 @@ kernel against the measured peaks, the CPU oracle's throughput on a bounded
 sample, and an end-to-end figure through the C ABI with host buffers.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
-and cudaDeviceSynchronize on both sides, replayed from CUDA graphs that hold
-the steps' C-ABI launches; CUDA events on the replay stream; per-kernel
-durations from external events captured between the kernels.  With N GPUs
+and a device synchronize on both sides, replayed from CUDA graphs that hold
+the steps' C-ABI launches; CUDA events on the replay stream (one between
+consecutive replays for the step-time percentiles).  The dominant kernel's
+duration (and the row gather's, for a top-k step) is timed the same way on
+graphs of 20 back-to-back launches of that kernel alone.  With N GPUs
 (torchrun) every rank runs its own replica of the workload and the time is
-the max over ranks.  Inputs are larger than L2 for the decode
-workloads (the KV cache alone is 302 MB vs 126 MB L2).
+the max over ranks.  Inputs are larger than L2 for the decode workloads (the
+KV cache alone is 302 MB vs 126 MB L2).  Other workloads: --workload
+gqa_decode, mla_decode, gqa_extend, mla_topk_decode, mqa_prefill,
+gqa_prefill, mla_prefill, mqa_prefill_tiny.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
