@@ -238,6 +238,29 @@ def test_brute_force_tiny_causal_gqa(impl):
                 assert abs(lse[b, h, i] - math.log(Z)) < 1e-13
 
 
+@pytest.mark.parametrize("impl", IMPLS)
+def test_extend_equals_token_by_token_decode(impl):
+    """Bottom-right alignment is what makes a chunk of Sq new tokens against
+    a cache the same as decoding them one at a time: query i of the chunk
+    equals a single decode query against the first skv - Sq + i + 1 keys
+    (decode itself is pinned to SDPA above).  Includes skv < Sq, where the
+    first queries see no key at all."""
+    B, Hq, Hkv, Sq, d, dv = 3, 4, 2, 4, 8, 6
+    q, k, v = rnd((B, Hq, Sq, d), 41), rnd((B, Hkv, 12, d), 42), rnd((B, Hkv, 12, dv), 43)
+    skv = [12, 4, 2]
+    out, lse = run(impl, q, k, v, skv, 0.6, True)
+    for b, L in enumerate(skv):
+        for i in range(Sq):
+            n = L - Sq + i + 1  # keys in the cache when token i arrives
+            if n <= 0:
+                assert (out[b, :, i] == 0).all() and np.isneginf(lse[b, :, i]).all()
+                continue
+            o1, l1 = run(impl, q[b:b + 1, :, i:i + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n],
+                         [n], 0.6, True)
+            np.testing.assert_allclose(out[b, :, i], o1[0, :, 0], rtol=1e-13, atol=1e-14)
+            np.testing.assert_allclose(lse[b, :, i], l1[0, :, 0], rtol=1e-13, atol=1e-14)
+
+
 # ----------------------------------------------------------------- MLA
 
 def test_mla_absorption_identity():
