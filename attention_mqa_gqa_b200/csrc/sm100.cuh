@@ -177,7 +177,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 4-D tiled TMA load (no multicast) into shared memory, completing on `bar`.
+// 4-D tiled TMA load into this CTA's shared memory, completing on `bar`.
 // Coordinates are element indices, innermost first; out-of-range parts of the
 // box are zero-filled.  c0 * element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -190,7 +190,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 5-D tiled TMA load (no multicast), same conventions as tma_load_4d.
+// 5-D tiled TMA load, same conventions as tma_load_4d.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, int c3, int c4,
                                             uint64_t policy) {
@@ -202,7 +202,7 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 3-D tiled TMA load (no multicast), same conventions as tma_load_4d.
+// 3-D tiled TMA load, same conventions as tma_load_4d.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, uint64_t policy) {
   asm volatile(
@@ -462,7 +462,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // Primitives for kernels launched as clusters of two CTAs on two SMs whose
 // UMMAs run as one (cta_group::2: M = 256 split 128/128 across the pair,
 // the B operand's N columns split half/half, one thread of the even CTA
-// issuing).  No load here uses cluster multicast.
+// issuing).  Every copy lands in the issuing CTA's own shared memory.
 namespace attn {
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -611,7 +611,7 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
       : "memory");
 }
 
-// Tiled TMA loads (no multicast) into this CTA's shared memory whose
+// Tiled TMA loads into this CTA's own shared memory whose
 // completion bytes are counted on an mbarrier of the even CTA of the pair
 // (`bar` is that barrier's shared::cluster address).
 __device__ __forceinline__ void tma_load_5d_pair(uint32_t dst, const CUtensorMap* map,
