@@ -52,3 +52,22 @@ def test_topk_accounting():
     assert w.is_decode
     assert bench.keys_of(w, inp).tolist() == [2048, 100, 2048]
     assert bench.kv_bytes(w, bench.keys_of(w, inp)) == (2048 + 100 + 2048) * 576 * 2
+
+
+def test_reference_arm_topk(monkeypatch, capsys):
+    """`bench.py --impl reference` on a top-k workload: the numpy top-k oracle
+    timed on the host, counted by the selected rows (a small instance of the
+    mla_topk_decode recipe)."""
+    import types
+
+    small = wl.WORKLOADS["mla_topk_decode"].scaled(name="topk_small", B=2, Hq=16, skv_lo=300,
+                                                   skv_hi=700, topk=128)
+    monkeypatch.setitem(wl.WORKLOADS, "topk_small", small)
+    args = types.SimpleNamespace(workload="topk_small", steps=1, warmup=0, ref_step_budget=0.5,
+                                 gpus=1)
+    assert bench.reference_arm(args, 1, 0) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["config"]["topk"] == 128 and "top-k" in line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
