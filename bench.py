@@ -33,6 +33,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -162,7 +163,7 @@ class ClockSampler:
 
     def __init__(self, device):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"attn_bench_clocks_{os.getpid()}.csv")
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
@@ -200,6 +201,10 @@ class ClockSampler:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) >= 9:
                     rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not rows:
             return None
         mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]

@@ -71,3 +71,27 @@ def test_reference_arm_topk(monkeypatch, capsys):
     assert line["config"]["topk"] == 128 and "top-k" in line["cpu_baseline"]["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_clock_sampler_summary(tmp_path):
+    """The clocks summary in the bench line: median SM MHz under load, the
+    maximum, and every throttle reason seen active (parsed from the
+    nvidia-smi CSV the sampler records; the sample file is removed)."""
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.path = str(tmp_path / "clocks.csv")
+    with open(cs.path, "w") as f:
+        f.write("0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+        f.write("0, 1900, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+
+    class _Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            pass
+
+    cs.proc, cs.f = _Proc(), open(os.devnull, "w")
+    assert cs.stop() == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                         "samples": 3}
+    assert not os.path.exists(cs.path)
