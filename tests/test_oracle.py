@@ -12,6 +12,8 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from oracle import attention as npo
 from oracle import c_oracle
@@ -424,3 +426,27 @@ def test_topk_rejects_positions_outside_the_sequence():
         npo.topk_attention_fwd(q, k, v, [10], np.array([[3, 10]]), [2], 0.5)
     with pytest.raises(ValueError):
         npo.topk_attention_fwd(q, k, v, [10], np.array([[-1, 2]]), [2], 0.5)
+
+
+# --------------------------------------------- the two oracles, randomised
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 3), Hkv=st.integers(1, 3), G=st.integers(1, 4), Sq=st.integers(1, 9),
+       d=st.sampled_from([1, 3, 8, 16]), dv=st.sampled_from([1, 5, 8]), causal=st.booleans(),
+       data=st.data())
+def test_numpy_and_c_oracles_agree(B, Hkv, G, Sq, d, dv, causal, data):
+    """The numpy and C oracles share no code; on random ragged shapes
+    (lengths 0..20, Sq above and below them, any grouping) they must agree
+    to rounding, including which rows are empty."""
+    skv = data.draw(st.lists(st.integers(0, 20), min_size=B, max_size=B))
+    S = max(max(skv), 1)
+    seed = data.draw(st.integers(0, 10_000))
+    q, k, v = rnd((B, Hkv * G, Sq, d), seed), rnd((B, Hkv, S, d), seed + 1), rnd((B, Hkv, S, dv), seed + 2)
+    scale = data.draw(st.sampled_from([0.1, 0.5, 1.3]))
+    o1, l1 = npo.attention_fwd(q, k, v, skv, scale, causal)
+    o2, l2 = c_oracle.attention_fwd(q, k, v, skv, scale, causal, nthreads=2)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    assert (np.isneginf(l1) == np.isneginf(l2)).all()
+    fin = np.isfinite(l1)
+    np.testing.assert_allclose(l1[fin], l2[fin], rtol=1e-12, atol=1e-13)
