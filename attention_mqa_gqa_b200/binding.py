@@ -168,11 +168,12 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    rc = fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                 lse.data_ptr() if lse is not None else None,
-                 B, Hq, Hkv, Sq, skv.data_ptr(), int(max_skv), d_k, d_v, scale, causal,
-                 dtype_code(q.dtype), _strides4(q), _strides4(k), _strides4(v), _strides4(out),
-                 ws_ptr, ws_n, st.cuda_stream)
+    with torch.cuda.device(q.device):  # the launch plan is made for the current device
+        rc = fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                     lse.data_ptr() if lse is not None else None,
+                     B, Hq, Hkv, Sq, skv.data_ptr(), int(max_skv), d_k, d_v, scale, causal,
+                     dtype_code(q.dtype), _strides4(q), _strides4(k), _strides4(v),
+                     _strides4(out), ws_ptr, ws_n, st.cuda_stream)
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
 
@@ -192,11 +193,12 @@ def attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: tor
         raise TypeError("lse must be a contiguous float32 tensor")
     _on_one_gpu(q, k, v, out, skv, lse)
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = load().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq,
-                                 skv.data_ptr(), int(max_skv), d_k, d_v, float(scale), int(causal),
-                                 dtype_code(q.dtype), _strides4(q), _strides4(k), _strides4(v),
-                                 _strides4(out), st.cuda_stream)
+    with torch.cuda.device(q.device):  # the library takes its scratch from the current device
+        rc = load().attn_fwd_noalloc(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+            lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq, skv.data_ptr(),
+            int(max_skv), d_k, d_v, float(scale), int(causal), dtype_code(q.dtype),
+            _strides4(q), _strides4(k), _strides4(v), _strides4(out), st.cuda_stream)
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_noalloc")
 

@@ -659,10 +659,12 @@ uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
 // code cannot pass the array's name to a kernel (on the host it only names a
 // stand-in object), so its device address is looked up once per device with
 // cudaGetSymbolAddress, with that device current, on the first call made on
-// that device.  All calls share the buffer and it keeps whatever the last
-// call left there; the kernels write every scratch value before reading it,
-// so nothing has to be cleared between calls.  Calls that overlap on the GPU
-// (other streams, other host threads) race on the buffer.
+// that device (and looked up again if the device's context has been
+// replaced since, e.g. after cudaDeviceReset).  All calls share the buffer
+// and it keeps whatever the last call left there; the kernels write every
+// scratch value before reading it, so nothing has to be cleared between
+// calls.  Calls that overlap on the GPU (other streams, other host threads)
+// race on the buffer.
 // ---------------------------------------------------------------------------
 
 namespace {
@@ -672,20 +674,44 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current CUDA context (null if it cannot be told).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_noalloc_scratch on the current device: looked up on
+// the first call on the device and again whenever the device's context is
+// not the one the cached address was taken in.
 attn_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return ATTN_ECUDA; }
   if (dev < 0 || dev >= kMaxDevices) return ATTN_EUNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  CUcontext ctx = current_context();
+  if (!g_noalloc_ptr[dev] || !ctx || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return ATTN_ECUDA;
     }
     g_noalloc_ptr[dev] = p;
+    // the lookup makes the device's primary context current if none was
+    g_noalloc_ctx[dev] = ctx ? ctx : current_context();
   }
   *out = g_noalloc_ptr[dev];
   return ATTN_OK;

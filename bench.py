@@ -7,15 +7,19 @@ Default workload: MQA decode at head_dim 512 (B=32, Hq=16, Hkv=1, per-sequence
 KV length uniform in [1024, 8192], bf16): one step = one decode forward of
 the whole batch (split-KV partial kernel + LSE combine).  The metric is the
 KV-cache bytes read per second (each cached K/V byte counted once).  The
-same line carries, measured in the same run, the d=512 MQA causal prefill
-(B=2, Hq=16, S=4096) in TFLOP/s, the roofline fraction of the dominant
-kernel against the measured peaks, the CPU oracle's throughput on a bounded
-sample, and an end-to-end figure through the C ABI with host buffers.
+same line carries, measured in the same run and each in an object of its
+own: the d=512 MQA causal prefill (B=2, Hq=16, S=4096; key "prefill"),
+absorbed-MLA decode ("mla_decode"), GQA d=128 decode ("gqa_decode") and GQA
+causal prefill ("gqa_prefill") -- each with its dominant kernel's roofline
+fraction against the measured and the datasheet peaks, the prefill ones with
+the CPU oracle on a sample -- plus the CPU oracle's throughput on a bounded
+sample of the main workload and an end-to-end figure through the C ABI with
+host buffers.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
-and a device synchronize on both sides, replayed from CUDA graphs that hold
-the steps' C-ABI launches; CUDA events on the replay stream (one between
-consecutive replays for the step-time percentiles).  The dominant kernel's
+and a device synchronize on both sides, replayed from CUDA graphs of two
+steps that hold the steps' C-ABI launches; CUDA events on the replay stream
+(one between consecutive replays for the step-time percentiles).  The dominant kernel's
 duration (and the row gather's, for a top-k step) is timed the same way on
 graphs of 20 back-to-back launches of that kernel alone.  With N GPUs
 (torchrun) every rank runs its own replica of the workload and the time is
@@ -54,6 +58,8 @@ KERNEL_SOURCES = {
     "gather_rows_kernel": [_CSRC + "sm100.cuh", _CSRC + "gather_rows.cuh", _CSRC + "attn_api.cu"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures: ~8 TB/s HBM3e, 2.25 PFLOP/s dense bf16/fp16 (no sparsity)
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 # ----------------------------------------------------------------- accounting
@@ -217,6 +223,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm
 
+def steps_per_graph(steps: int) -> int:
+    """Steps captured in one CUDA graph: two (one if K is odd), so that K
+    timed steps give K/2 replays and the step-time percentiles come from
+    many samples rather than one."""
+    return 2 if steps % 2 == 0 else 1
+
+
 class GpuRunner:
     """Holds one workload's device tensors and launches steps through the C ABI."""
 
@@ -330,14 +343,14 @@ class GpuRunner:
 
     def timed(self, steps, warmup):
         """Warm up, then time exactly `steps` steps replayed from CUDA graphs
-        (captured `per` steps at a time); CUDA events on the replay stream.
+        (captured two steps at a time); CUDA events on the replay stream.
         Returns (total_ms, dominant kernel mean ms, other kernel mean ms).
         The dominant kernel's duration is timed the same way over graphs of
         20 back-to-back launches of that kernel alone (for decode the split
         kernel, whose inputs do not depend on the combine); the combine's is
         the step time minus that (and minus the row gather of a top-k step,
         timed the same way, in ``self.gather_ms``)."""
-        per = max(d for d in range(1, min(steps, 20) + 1) if steps % d == 0)
+        per = steps_per_graph(steps)
         graph, side = self._graph(per)
         reps = []
         total = self._replay_ms(graph, side, steps // per, max(1, warmup // per), reps)
@@ -418,28 +431,40 @@ def value_of(w, skv, ms):
 
 
 def roofline(w, skv, kernel_ms, peaks, peak_src, long_run, traffic):
+    """Roofline of the dominant kernel: `frac` against the measured peak of
+    this machine's B200s (MEASURED_PEAKS.json, else the fallback figures), and
+    `frac_nominal` against the datasheet figure (~8 TB/s HBM, 2.25 PFLOP/s
+    dense bf16), each labelled with its denominator."""
     if w.is_decode:
         achieved = kv_bytes(w, skv) / (kernel_ms * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
+        nom = NOMINAL_PEAKS["hbm_gbs"]
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": f"hbm_gbs ({peak_src})"}
+                "peak_source": f"hbm_gbs ({peak_src})",
+                "peak_nominal": nom, "frac_nominal": round(achieved / nom, 4),
+                "peak_nominal_source": "B200 datasheet HBM3e ~8 TB/s"}
     key = "bf16_tflops_sustained" if long_run else "bf16_tflops"
     peak = float(peaks[key])
     if w.dtype == torch.float16:
         key += " (fp16 = bf16 dense rate)"
     achieved = flops(w, skv) / (kernel_ms * 1e-3) / 1e12
+    nom = NOMINAL_PEAKS["bf16_tflops"]
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "peak_source": f"{key} ({peak_src})"}
+            "peak_source": f"{key} ({peak_src})",
+            "peak_nominal": nom, "frac_nominal": round(achieved / nom, 4),
+            "peak_nominal_source": "B200 datasheet dense bf16/fp16 2.25 PFLOP/s"}
 
 
-def config_of(w, inp, parallelism):
+def config_of(w, inp):
+    """The workload (the same for the GPU arm and the reference arm; where it
+    runs is reported beside it, in the line's `parallelism`)."""
     skv = inp["skv"]
     d = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "d_k": w.d_k,
          "d_v": w.d_v, "causal": w.causal, "scale": round(w.scale, 6), "mla_absorbed": w.mla,
          "skv": f"U[{w.skv_lo},{w.skv_hi}] seed {w.seed}" if w.skv_lo != w.skv_hi else w.skv_lo,
-         "skv_total": int(skv.sum()), "parallelism": parallelism}
+         "skv_total": int(skv.sum())}
     if w.topk:
         sel = kv_bytes(w, inp["n_sel"])
         d["topk"] = w.topk
@@ -562,7 +587,7 @@ def reference_arm(args, world, rank):
             "unit": unit, "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": round(t / steps * 1e3, 3), "higher_is_better": hib,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, inp, "host cores"),
+            "config": config_of(w, inp), "parallelism": f"host cores x{cores}",
             "cpu_baseline": {"value": round(val, 4), "unit": unit, "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(val, 4), "unit": unit, "h2d_bytes_per_step": 0,
@@ -586,6 +611,103 @@ def measure_workload(w, inp, device, steps, warmup, world):
     return g, steps, total_ms, k_ms, other_ms, clocks
 
 
+def step_dist_of(g, steps):
+    samples = sorted(g.step_ms_samples)
+    pct = lambda q: samples[min(len(samples) - 1, int(q * (len(samples) - 1) + 0.5))]
+    return {"p10": round(pct(0.1), 5), "p50": round(pct(0.5), 5), "p90": round(pct(0.9), 5),
+            "replays": len(samples), "steps_per_replay": steps // len(samples)}
+
+
+def kernel_name(w, g):
+    if not g.decode:
+        return "prefill_kernel"
+    return "mla_pair_kernel" if w.mla else "decode_split_kernel"
+
+
+def dominant_roofline(w, g, keys, k_ms, other_ms, total_ms, peaks, peak_src):
+    kname = kernel_name(w, g)
+    roof = roofline(w, keys, k_ms, peaks, peak_src, total_ms > 1000.0, traffic_for(kname, w.name))
+    roof["kernel"] = kname
+    roof["kernel_ms"] = round(k_ms, 5)
+    if g.decode:
+        roof["combine_ms"] = round(other_ms, 5)
+    return roof
+
+
+def cpu_leg(w, inp, budget_s, one_core=True):
+    """The fp64 C oracle (numpy for top-k) as it stands, on a bounded sample of
+    the workload, on all host cores and (if asked) on one thread."""
+    from oracle import c_oracle
+
+    c_oracle.build()
+    cores = os.cpu_count() or 1
+    metric, unit, _ = metric_of(w)
+    which = "numpy fp64 top-k oracle" if w.topk else "fp64 C oracle"
+    if w.is_decode:
+        n = oracle_sample(w, inp, budget_s=budget_s)
+        secs = run_oracle(w, inp, n)
+        d = {"value": round(cpu_value(w, inp, n, secs), 4), "unit": unit, "cores": cores,
+             "kind": "oracle",
+             "sample": f"first {n} of {w.B} sequences, all {w.Hq} heads ({secs:.1f} s, {which})"}
+        if one_core and not w.topk:  # the same oracle on one host thread, first sequence
+            s1 = run_oracle(w, inp, 1, nthreads=1)
+            d["value_1core"] = round(cpu_value(w, inp, 1, s1), 4)
+            d["sample_1core"] = f"first sequence, all {w.Hq} heads, one thread ({s1:.2f} s)"
+        return d
+    # prefill: the oracle threads over (sequence, query head); one head per
+    # host thread, every query row of each
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hq)][:cores]
+    work = flops(w.scaled(B=1, Hq=1), inp["skv"][:1].tolist())  # one head's FLOPs
+    t0 = time.perf_counter()
+    c_oracle.attention_fwd(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(), w.scale, w.causal,
+                           pairs=pairs)
+    secs = time.perf_counter() - t0
+    d = {"value": round(work * len(pairs) / secs / 1e12, 6), "unit": unit, "cores": cores,
+         "kind": "oracle",
+         "sample": f"{len(pairs)} of {w.B * w.Hq} (sequence, head) pairs, every query row "
+                   f"({secs:.1f} s, {which})"}
+    if one_core:
+        t0 = time.perf_counter()
+        c_oracle.attention_fwd(inp["q"], inp["k"], inp["v"], inp["skv"].tolist(), w.scale,
+                               w.causal, nthreads=1, pairs=pairs[:1])
+        s1 = time.perf_counter() - t0
+        d["value_1core"] = round(work / s1 / 1e12, 6)
+        d["sample_1core"] = f"one (sequence, head) pair, every query row, one thread ({s1:.2f} s)"
+    return d
+
+
+# Workloads whose figures the default line carries beside its own (key in
+# the line: workload), each measured in the same run the same way.
+SECONDARY = (("prefill", "mqa_prefill"), ("mla_decode", "mla_decode"),
+             ("gqa_decode", "gqa_decode"), ("gqa_prefill", "gqa_prefill"))
+
+
+def secondary(name, rank, world, device, args, peaks, peak_src, with_cpu):
+    import torch.distributed as dist_mod
+
+    w = wl.WORKLOADS[name]
+    if rank:
+        w = w.scaled(seed=w.seed + 1000 * rank)
+    inp = wl.make_inputs(w)
+    g, steps, tot, k_ms, other_ms, clocks = measure_workload(w, inp, device, args.steps,
+                                                             args.warmup, world)
+    mx = allreduce(tot, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
+    keys = keys_of(w, inp)
+    work = kv_bytes(w, keys) if w.is_decode else flops(w, keys)
+    work = allreduce(work, dist_mod.ReduceOp.SUM if world > 1 else None, world, device)
+    metric, unit, _ = metric_of(w)
+    scale_div = 1e9 if w.is_decode else 1e12
+    d = {"metric": f"{w.name}_{metric}", "value": round(work * steps / (mx * 1e-3) / scale_div, 3),
+         "unit": unit, "steps": steps, "ms_per_step": round(mx / steps, 5),
+         "ms_per_step_dist": step_dist_of(g, steps), "config": config_of(w, inp),
+         "roofline": dominant_roofline(w, g, keys, k_ms, other_ms, tot, peaks, peak_src),
+         "gpu_launches": g.launches_per_step() * steps, "clocks": clocks}
+    del g
+    if with_cpu and not w.is_decode:
+        d["cpu_baseline"] = cpu_leg(w, inp, budget_s=10.0)
+    return d
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -593,7 +715,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mqa_decode", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill figure")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' figures in the default line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--ref-step-budget", type=float, default=2.0)
     args = ap.parse_args()
@@ -633,17 +756,7 @@ def main():
     scale_div = 1e9 if w.is_decode else 1e12
     value = work_all * steps / (max_ms * 1e-3) / scale_div
     metric, unit, hib = metric_of(w)
-    long_run = total_ms > 1000.0
-    kname = ("mla_pair_kernel" if w.mla else "decode_split_kernel") if g.decode else "prefill_kernel"
-    samples = sorted(g.step_ms_samples)
-    pct = lambda q: samples[min(len(samples) - 1, int(q * (len(samples) - 1) + 0.5))]
-    step_dist = {"p10": round(pct(0.1), 5), "p50": round(pct(0.5), 5), "p90": round(pct(0.9), 5),
-                 "replays": len(samples), "steps_per_replay": steps // len(samples)}
-    roof = roofline(w, keys, k_ms, peaks, peak_src, long_run, traffic_for(kname, w.name))
-    roof["kernel"] = kname
-    roof["kernel_ms"] = round(k_ms, 5)
-    if g.decode:
-        roof["combine_ms"] = round(other_ms, 5)
+    roof = dominant_roofline(w, g, keys, k_ms, other_ms, total_ms, peaks, peak_src)
     if w.topk:  # the row gather: reads and writes the selected rows once each
         gb = 2 * kv_bytes(w, keys) / (g.gather_ms * 1e-3) / 1e9
         roof["gather"] = {"kernel": "gather_rows_kernel", "ms": round(g.gather_ms, 5),
@@ -660,54 +773,27 @@ def main():
 
     line = {"metric": f"{w.name}_{metric}", "value": round(value, 3), "unit": unit,
             "n_gpus": world, "steps": steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_step, 5), "ms_per_step_dist": step_dist,
+            "ms_per_step": round(ms_step, 5), "ms_per_step_dist": step_dist_of(g, steps),
             "higher_is_better": hib, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "fp16",
             "data": "synthetic (seeded N(0,1), rounded once to the element type)",
-            "config": config_of(w, inp, f"replicas x{world}" if world > 1 else "single GPU"),
+            "config": config_of(w, inp),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "roofline": roof, "gpu_launches": g.launches_per_step() * steps,
             "clocks": clocks,
             "e2e": {"value": round(e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps}}
     del g
 
-    # secondary figure: d=512 MQA causal prefill (B=2, Hq=16, S=4096)
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu
     if not args.no_secondary and args.workload == "mqa_decode":
-        w2 = wl.WORKLOADS["mqa_prefill"]
-        if rank:
-            w2 = w2.scaled(seed=w2.seed + 1000 * rank)
-        inp2 = wl.make_inputs(w2)
-        g2, steps2, tot2, k2, _, clocks2 = measure_workload(w2, inp2, device, args.steps,
-                                                            args.warmup, world)
-        max2 = allreduce(tot2, dist_mod.ReduceOp.MAX if world > 1 else None, world, device)
-        work2 = allreduce(flops(w2, inp2["skv"]), dist_mod.ReduceOp.SUM if world > 1 else None,
-                          world, device)
-        r2 = roofline(w2, inp2["skv"], k2, peaks, peak_src, tot2 > 1000.0,
-                      traffic_for("prefill_kernel", w2.name))
-        r2["kernel"] = "prefill_kernel"
-        line["prefill"] = {"metric": f"{w2.name}_attention_TFLOPs",
-                           "value": round(work2 * steps2 / (max2 * 1e-3) / 1e12, 2),
-                           "unit": "TFLOP/s", "steps": steps2, "ms_per_step": round(max2 / steps2, 4),
-                           "config": config_of(w2, inp2, "single GPU" if world == 1 else f"replicas x{world}"),
-                           "roofline": r2, "clocks": clocks2}
-        del g2
+        for key, name in SECONDARY:
+            line[key] = secondary(name, rank, world, device, args, peaks, peak_src, with_cpu)
+            torch.cuda.empty_cache()
+        assert binding.last_device_error() == binding.ATTN_OK, "device-side wait timed out"
 
-    if rank == 0 and world == 1 and not args.no_cpu:
-        n = oracle_sample(w, inp, budget_s=15.0)
-        from oracle import c_oracle
-
-        c_oracle.build()
-        secs = run_oracle(w, inp, n)
-        which = "numpy fp64 top-k oracle" if w.topk else "fp64 C oracle"
-        line["cpu_baseline"] = {"value": round(cpu_value(w, inp, n, secs), 4), "unit": unit,
-                                "cores": os.cpu_count() or 1, "kind": "oracle",
-                                "sample": f"first {n} of {w.B} sequences, all {w.Hq} heads "
-                                          f"({secs:.1f} s, {which})"}
-        if not w.topk:  # the same oracle on one host thread, first sequence
-            s1 = run_oracle(w, inp, 1, nthreads=1)
-            line["cpu_baseline"]["value_1core"] = round(cpu_value(w, inp, 1, s1), 4)
-            line["cpu_baseline"]["sample_1core"] = (f"first sequence, all {w.Hq} heads, one thread "
-                                                    f"({s1:.2f} s)")
+    if with_cpu:
+        line["cpu_baseline"] = cpu_leg(w, inp, budget_s=15.0)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

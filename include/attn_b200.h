@@ -173,12 +173,15 @@ attn_status_t attn_decode_combine(const void* q, const void* k, const void* v, v
  * the library (held on every GPU that loads the library until the process
  * exits); the call itself allocates nothing.  Problems whose scratch
  * (attn_workspace_bytes) exceeds that size return ATTN_EWORKSPACE before
- * anything is enqueued.  The first call on each device looks up the
- * buffer's device address (cudaGetSymbolAddress, that device current); make
- * that first call before any stream capture.  All calls share the buffer:
- * calls that overlap on the GPU (concurrent streams or host threads) race,
- * so serialise them.  Otherwise the same arguments, semantics and errors as
- * attn_fwd.
+ * anything is enqueued.  The device that holds the tensors and owns
+ * `cuda_stream` must be the calling thread's current device: the buffer
+ * and the launch plan are taken from the current device.  The first call
+ * on each device looks up the buffer's device address (cudaGetSymbolAddress,
+ * that device current), and so does the first call after the device's
+ * context has been replaced (cudaDeviceReset); make that first call before
+ * any stream capture.  All calls share the buffer: calls that overlap on
+ * the GPU (concurrent streams or host threads) race, so serialise them.
+ * Otherwise the same arguments, semantics and errors as attn_fwd.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
 attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,

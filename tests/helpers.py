@@ -3,14 +3,18 @@ and compare it with the fp64 oracle under one tolerance.
 
 Tolerance (elementwise): |gpu - oracle| <= 1e-2 + 1e-2 * |oracle| for the
 output and |gpu_lse - oracle_lse| <= 1e-3 for the log-sum-exp (rows with
-no visible key must give exactly 0 and -inf).
+no visible key must give exactly 0 and -inf).  Because long-context outputs
+are small averages (|O| ~ 0.02-0.05) the absolute term alone would admit
+gross errors, so the relative Frobenius error ||gpu - oracle|| / ||oracle||
+over everything compared must also stay within 1e-2 (bf16 rounding of P and
+of the output contribute about 3e-3).
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-ATOL, RTOL, LSE_TOL = 1e-2, 1e-2, 1e-3
+ATOL, RTOL, LSE_TOL, REL_FRO = 1e-2, 1e-2, 1e-3, 1e-2
 
 
 def to_device(inp: dict, device="cuda") -> dict:
@@ -66,4 +70,5 @@ def compare(out_gpu, lse_gpu, ref_o, ref_l, what=""):
         assert (o[empty] == 0).all(), f"{what}: rows with no visible key must be 0"
     den = np.linalg.norm(ref_o)
     rel = float(np.linalg.norm(o - ref_o) / den) if den > 0 else 0.0
+    assert rel <= REL_FRO, f"{what}: relative Frobenius error {rel:.3e}"
     return float(err.max()), lerr, rel

@@ -71,6 +71,33 @@ def test_reference_arm_topk(monkeypatch, capsys):
     assert line["config"]["topk"] == 128 and "top-k" in line["cpu_baseline"]["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+    # the reference arm names the same workload as the GPU arm: where each
+    # runs is reported outside `config`
+    inp = wl.make_inputs(small)
+    assert line["config"] == bench.config_of(small, inp)
+    assert "parallelism" not in line["config"] and line["parallelism"].startswith("host cores")
+
+
+def test_timed_steps_give_many_replays():
+    """20 timed steps are replayed as 10 graphs of two steps (K odd: one step
+    per graph), so the step-time percentiles rest on many samples."""
+    for k in (20, 100, 2):
+        assert bench.steps_per_graph(k) == 2 and k // bench.steps_per_graph(k) == k // 2
+    assert bench.steps_per_graph(21) == 1
+
+
+def test_roofline_reports_measured_and_nominal_fractions():
+    w = wl.WORKLOADS["mqa_decode"]
+    skv = [1000, 3000]
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1300.0}
+    ms = bench.kv_bytes(w, skv) / 4.0e12 * 1e3  # 4 TB/s
+    r = bench.roofline(w, skv, ms, peaks, "measured", False, None)
+    assert abs(r["frac"] - 4000 / 6000) < 1e-3 and abs(r["frac_nominal"] - 0.5) < 1e-3
+    assert r["peak_nominal"] == 8000.0 and r["bound"] == "hbm"
+    wp = wl.WORKLOADS["mqa_prefill"]
+    ms = bench.flops(wp, [4096, 4096]) / 1.125e15 * 1e3  # 1125 TFLOP/s
+    r = bench.roofline(wp, [4096, 4096], ms, peaks, "measured", True, None)
+    assert abs(r["frac"] - 1125 / 1300) < 1e-3 and abs(r["frac_nominal"] - 0.5) < 1e-3
 
 
 def test_clock_sampler_summary(tmp_path):

@@ -32,6 +32,14 @@ def test_header_declarations_are_exported(lib):
         assert hasattr(lib, n), f"{n} declared in the header but not exported"
 
 
+def test_noalloc_scratch_size_matches_header():
+    """The binding's copy of the built-in scratch size is the header's."""
+    m = re.search(r"#define\s+ATTN_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)",
+                  open(HEADER).read())
+    assert m, "ATTN_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert binding.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert binding.status_str(code) and binding.status_str(code) != "unknown status"

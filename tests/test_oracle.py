@@ -336,7 +336,9 @@ def test_byte_model_matches_printed_tables():
         assert npo.kv_bytes_per_token(row["kind"], **kw) == row["bytes"]
     cd = g["cache_dims_per_token"]
     assert npo.kv_bytes_per_token("mha", elem_bytes=1) == cd["mha_values"]
-    assert 512 == cd["mla_values"]
+    # the p5 table counts only the latent c_kv values (no rope part), one element each
+    assert npo.kv_bytes_per_token("mla", d_R=0, elem_bytes=1) == cd["mla_values"]
+    assert cd["mha_values"] / cd["mla_values"] == 64  # the page's ~64x reduction
     mq = g["mqa_cache_fraction"]
     assert npo.kv_bytes_per_token("mqa", d_h=512) / npo.kv_bytes_per_token(
         "mha", H=mq["query_heads"], d_h=512) == mq["fraction"]
