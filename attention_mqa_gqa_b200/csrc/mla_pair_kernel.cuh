@@ -16,8 +16,8 @@
 //       split by heads: CTA r holds heads 64r..64r+63.  Each CTA's TMEM gets
 //       S^T of its own 128 keys for all 128 heads.
 //   softmax over keys per head: each CTA reduces its 128 keys, the two CTAs
-//       exchange per-head tile maxima through distributed shared memory so
-//       that both use the same running maximum.
+//       exchange per-head tile maxima (st.async into the other CTA's shared
+//       memory) so that both use the same running maximum.
 //   O^T[512 x 128] += V^T[512 x 256 keys] * P^T[256 keys x 128 heads]
 //       two pair MMAs (d rows 0..255 and 256..511, M = 256): CTA r provides
 //       d rows 256m + 128r .. +127 of block m (two 64-column chunks of V for
@@ -33,10 +33,16 @@
 //
 // Roles (320 threads per CTA): warp 0 lane 0 streams K/V groups, lane 1
 // loads this CTA's Q^T half per piece; warp 1 allocates the pair's TMEM and,
-// in CTA 0 only, issues the pair UMMAs; warps 2-9 run the softmax (two
-// threads per key row, 64 heads each) and the epilogue.  All waits are
-// bounded; the CTAs meet in a hardware cluster barrier only after both have
-// left every loop.
+// in CTA 0, issues the pair UMMAs, in CTA 1 tells CTA 0 when its P^T buffer
+// is complete; warps 2-9 run the softmax (two threads per key row, 64 heads
+// each) and the epilogue.  All waits are bounded; the CTAs meet in a
+// hardware cluster barrier only after both have left every loop.
+//
+// Cross-CTA traffic avoids cluster-scope release arrivals, which stall the
+// arriving thread for about a microsecond while the SM streams copies: data
+// (tile maxima, row sums, P^T rows) goes by st.async, whose bytes complete
+// an mbarrier of the receiving CTA; signals without data (S^T read) are
+// relaxed arrivals; MMA completions are tcgen05.commit multicasts.
 #pragma once
 
 #include "decode_kernel.cuh"
@@ -69,9 +75,10 @@ struct MlaPairTraits {
   static constexpr int OFF_SCHED = OFF_SCAN + 64;           // int [4]
   static constexpr int OFF_FLAGS = OFF_SCHED + 16;          // int [4]: any[2], abort, tmem
   static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
-  // full[3] empty[3] q_full q_free s_full[2] s_free[2] p_full o_done red_full[2]
-  // stat_ready[2] xmax_full[2] lsum_full drain
-  static constexpr int NBAR = 2 * RING_G + 2 + 2 + 2 + 1 + 1 + 2 + 2 + 2 + 1 + 1;
+  // full[3] empty[3] q_full q_free s_full[2] s_free[2] p_local p_recv p_peer o_done
+  // red_full[2] stat_ready[2] xmax_full[2] lsum_full drain
+  static constexpr int NBAR = 2 * RING_G + 2 + 2 + 2 + 3 + 1 + 2 + 2 + 2 + 1 + 1;
+  static constexpr int PT_PEER_BYTES = TILE * NHC * 2;     // P^T rows one CTA sends the other
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int SOFTMAX_THREADS = 256;
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
@@ -137,9 +144,11 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
   const uint32_t q_full = bar0 + 8u * (2 * T::RING_G);
   const uint32_t q_free = q_full + 8;
   const uint32_t s_full = q_free + 8;        // [2]
-  const uint32_t s_free = s_full + 16;       // [2] (CTA 0: both CTAs' softmax)
-  const uint32_t p_full = s_free + 16;       // CTA 0: both CTAs' P^T writes
-  const uint32_t o_done = p_full + 8;
+  const uint32_t s_free = s_full + 16;       // [2] (CTA 0: both CTAs' softmax warps)
+  const uint32_t p_local = s_free + 16;      // this CTA's own P^T rows written
+  const uint32_t p_recv = p_local + 8;       // the other CTA's P^T rows landed (st.async bytes)
+  const uint32_t p_peer = p_recv + 8;        // CTA 0: CTA 1's P^T buffer complete
+  const uint32_t o_done = p_peer + 8;
   const uint32_t red_full = o_done + 8;      // [2]
   const uint32_t stat_ready = red_full + 16; // [2]
   const uint32_t xmax_full = stat_ready + 16;  // [2] peer maxima landed
@@ -156,21 +165,27 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
+    constexpr int SW = T::SOFTMAX_THREADS / 32;  // softmax warps
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(s_free + 8 * i, 2 * T::SOFTMAX_THREADS);
-      mbar_init(red_full + 8 * i, T::SOFTMAX_THREADS);
-      mbar_init(stat_ready + 8 * i, NH);
-      mbar_init(xmax_full + 8 * i, NH);
+      mbar_init(s_free + 8 * i, 2 * SW);      // one arrival per softmax warp of each CTA
+      mbar_init(red_full + 8 * i, SW);
+      mbar_init(stat_ready + 8 * i, NH / 32);
+      mbar_init(xmax_full + 8 * i, 1);        // the local arm; the peer's bytes complete it
     }
-    mbar_init(p_full, 2 * T::SOFTMAX_THREADS);
+    mbar_init(p_local, SW / 2);               // the warps writing this CTA's own heads
+    mbar_init(p_recv, 1);
+    mbar_init(p_peer, 1);
     mbar_init(o_done, 1);
-    mbar_init(lsum_full, NH);
+    mbar_init(lsum_full, 1);
     mbar_init(drain, 1);
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
     fence_mbar_init();  // release at cluster scope
+    // the first tile's P^T rows from the other CTA (later tiles are armed by
+    // the thread that sees the previous phase complete)
+    mbar_arrive_expect_tx(p_recv, T::PT_PEER_BYTES);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), 512);
@@ -273,8 +288,15 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
       bool ok = true;
       auto pv = [&](int t, bool first_of_piece) {
         if (!ok) return;
-        ok = mbar_wait_warp_cluster(p_full, t & 1, abort_flag, p.timeout_ns, 43);
+        // P^T of tile t complete in both CTAs: this CTA's own rows, the rows
+        // CTA 1 sent here, and CTA 1's buffer (forwarded by CTA 1)
+        ok = mbar_wait_warp(p_local, t & 1, abort_flag, p.timeout_ns, 43) &&
+             mbar_wait_warp_cluster(p_recv, t & 1, abort_flag, p.timeout_ns, 48) &&
+             mbar_wait_warp_cluster(p_peer, t & 1, abort_flag, p.timeout_ns, 49);
         if (!ok) return;
+        if (elect_one()) mbar_arrive_expect_tx(p_recv, T::PT_PEER_BYTES);  // next tile's rows
+        __syncwarp();
+        fence_proxy_async_smem();  // the st.async rows, for the MMA's operand reads
         tc_fence_after();
         for (int m = 0; m < 2; ++m) {
           for (int h = 0; h < 2; ++h) {
@@ -359,6 +381,27 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
         ++k;
       }
       if (ok && j > 0) pv(j - 1, prev_first);
+    } else if (warp == 1) {
+      // ------------------------------------------------ CTA 1: P^T forwarder
+      // CTA 0's MMAs read this CTA's P^T buffer: once this CTA's own rows are
+      // written and the rows from CTA 0 have landed, tell CTA 0.
+      const uint32_t p_peer_lead = mapa_shared(p_peer, 0);
+      PieceWalker w = walker();
+      int b, kvh, t0, n, j = 0;
+      bool ok = true;
+      while (ok && w.next(b, kvh, t0, n)) {
+        for (int i = 0; i < n && ok; ++i, ++j) {
+          ok = mbar_wait_warp(p_local, j & 1, abort_flag, p.timeout_ns, 61) &&
+               mbar_wait_warp_cluster(p_recv, j & 1, abort_flag, p.timeout_ns, 62);
+          if (!ok) break;
+          if (elect_one()) mbar_arrive_expect_tx(p_recv, T::PT_PEER_BYTES);
+          __syncwarp();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (elect_one()) mbar_arrive_remote_cta(p_peer_lead);
+          __syncwarp();
+        }
+      }
     } else if (warp >= 2) {
       // ------------------------------------------------ softmax + epilogues
       constexpr int HH = NHC;                  // heads per thread (64)
@@ -369,13 +412,20 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
       const int row = wq * 32 + lane;          // key row of S^T / d row of O^T blocks
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
       volatile int own_abort = 0;
+      // barriers completed by the other CTA (arrivals, st.async bytes, pair
+      // commits) are waited on with cluster-scope acquire, local ones at CTA scope
       auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
         return mbar_wait_warp_cluster(bar, parity, &own_abort, p.timeout_ns, id);
       };
-      // where this thread's P^T row goes: its heads are CTA `half`'s columns
-      const uint32_t pdst = half == (int)cr ? pt : mapa_shared(pt, (uint32_t)half);
+      auto wait_l = [&](uint32_t bar, uint32_t parity, uint32_t id) {
+        return mbar_wait_warp(bar, parity, &own_abort, p.timeout_ns, id);
+      };
+      // where this thread's P^T row goes: its heads are CTA `half`'s columns;
+      // rows for the other CTA go by st.async, counted on that CTA's p_recv
+      const bool local_heads = half == (int)cr;
+      const uint32_t pdst = local_heads ? pt : mapa_shared(pt, (uint32_t)half);
+      const uint32_t p_recv_peer = mapa_shared(p_recv, peer);
       const uint32_t s_free_lead = mapa_shared(s_free, 0);
-      const uint32_t p_full_lead = mapa_shared(p_full, 0);
       if (st < NH) m_sm[st] = -INFINITY;
       named_bar_sync(1, T::SOFTMAX_THREADS);
 
@@ -414,8 +464,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < HH / 32; ++e) rbuf[wq * NH + h0l + transposed_head<HH>(lane, e)] = v[e];
           }
-          mbar_arrive(red_full + 8 * rb);
-          ok = wait(red_full + 8 * rb, rpar, 52);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(red_full + 8 * rb);
+          ok = wait_l(red_full + 8 * rb, rpar, 52);
           if (!ok) break;
           if (st == 0) flags[rb ^ 1] = 0;
           if (st < NH) {
@@ -423,8 +474,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
             // maximum over the pair tile's 256 keys
             const float own =
                 fmaxf(fmaxf(rbuf[st], rbuf[NH + st]), fmaxf(rbuf[2 * NH + st], rbuf[3 * NH + st]));
-            st_cluster_f32(mapa_shared(smem_u32(pmax_in + (j & 1) * NH + st), peer), own);
-            mbar_arrive_remote(mapa_shared(xmax_full + 8 * (j & 1), peer));
+            st_async_f32(mapa_shared(smem_u32(pmax_in + (j & 1) * NH + st), peer), own,
+                         mapa_shared(xmax_full + 8 * (j & 1), peer));
+            if (st == 0) mbar_arrive_expect_tx(xmax_full + 8 * (j & 1), NH * 4);  // the peer's maxima
             ok = wait(xmax_full + 8 * (j & 1), (j >> 1) & 1, 53);
             if (ok) {
               const float tm = fmaxf(own, pmax_in[(j & 1) * NH + st]);
@@ -436,10 +488,11 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
               m_sm[st] = mn;
               if (need) flags[rb] = 1;
             }
-            mbar_arrive(stat_ready + 8 * rb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stat_ready + 8 * rb);
           }
           if (!ok) break;
-          ok = wait(stat_ready + 8 * rb, rpar, 54);
+          ok = wait_l(stat_ready + 8 * rb, rpar, 54);
           if (!ok) break;
           const bool any = flags[rb] != 0;
 
@@ -498,10 +551,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
               const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
               for (int q = 0; q < 4; q += 2) {
-                const float x0 = valid ? sv[e + q] * p.scale_log2 : -INFINITY;
-                const float x1 = valid ? sv[e + q + 1] * p.scale_log2 : -INFINITY;
-                const float p0 = x0 == -INFINITY ? 0.f : ex2(x0 - mm[q]);
-                const float p1 = x1 == -INFINITY ? 0.f : ex2(x1 - mm[q + 1]);
+                // an invalid row's weights are exactly 0 (ex2(-inf) = +0)
+                const float p0 = valid ? ex2(fmaf(sv[e + q], p.scale_log2, -mm[q])) : 0.f;
+                const float p1 = valid ? ex2(fmaf(sv[e + q + 1], p.scale_log2, -mm[q + 1])) : 0.f;
                 u[(e + q) >> 1] = pack2(p0, p1, BF16);
                 l[c0 + e + q] += p0;
                 l[c0 + e + q + 1] += p1;
@@ -509,18 +561,26 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
             }
             const uint32_t a0 = prow + ((c0 >> 3) + 0) * 128;
             const uint32_t a1 = prow + ((c0 >> 3) + 1) * 128;
-            if (half == (int)cr) {
+            if (local_heads) {
               st_shared_v4(a0, u[0], u[1], u[2], u[3]);
               st_shared_v4(a1, u[4], u[5], u[6], u[7]);
             } else {
-              st_cluster_v4(a0, u[0], u[1], u[2], u[3]);
-              st_cluster_v4(a1, u[4], u[5], u[6], u[7]);
+              st_async_v4(a0, u[0], u[1], u[2], u[3], p_recv_peer);
+              st_async_v4(a1, u[4], u[5], u[6], u[7], p_recv_peer);
             }
           }
+          // S^T(j) has been read (a signal without data: CTA 1 arrives relaxed)
           tc_fence_before();
-          mbar_arrive_remote(s_free_lead + 8 * sb);  // S^T(j) has been read
-          fence_proxy_async_cluster();
-          mbar_arrive_remote(p_full_lead);
+          __syncwarp();
+          if (lane == 0) {
+            if (cr == 0) mbar_arrive(s_free + 8 * sb);
+            else mbar_arrive_remote_relaxed(s_free_lead + 8 * sb);
+          }
+          if (local_heads) {  // this CTA's own P^T rows, for the MMA's operand reads
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_local);
+          }
         }
         if (!ok) break;
 
@@ -536,14 +596,15 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
           transposed_warp_sum<HH, HH, 16>(l, lane);
 #pragma unroll
           for (int e = 0; e < HH / 32; ++e) rbuf[wq * NH + h0l + transposed_head<HH>(lane, e)] = l[e];
-          mbar_arrive(red_full + 8 * rb);
-          ok = wait(red_full + 8 * rb, rpar, 57);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(red_full + 8 * rb);
+          ok = wait_l(red_full + 8 * rb, rpar, 57);
           if (!ok) break;
           if (st == 0) flags[rb ^ 1] = 0;
           if (st < NH) {
             const float own = (rbuf[st] + rbuf[NH + st]) + (rbuf[2 * NH + st] + rbuf[3 * NH + st]);
-            st_cluster_f32(mapa_shared(smem_u32(lpeer + st), peer), own);
-            mbar_arrive_remote(mapa_shared(lsum_full, peer));
+            st_async_f32(mapa_shared(smem_u32(lpeer + st), peer), own, mapa_shared(lsum_full, peer));
+            if (st == 0) mbar_arrive_expect_tx(lsum_full, NH * 4);  // the peer's sums
             ok = wait(lsum_full, pc & 1, 58);
             if (ok) {
               // the same sum in both CTAs: CTA 0's keys first
@@ -554,10 +615,11 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
                     L > 0.f ? (m_sm[st] + __log2f(L)) * 0.69314718055994531f : -INFINITY;
               m_sm[st] = -INFINITY;  // the next piece starts afresh
             }
-            mbar_arrive(stat_ready + 8 * rb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stat_ready + 8 * rb);
           }
           if (!ok) break;
-          ok = wait(stat_ready + 8 * rb, rpar, 59);
+          ok = wait_l(stat_ready + 8 * rb, rpar, 59);
           if (!ok) break;
           ++r;
           ++pc;

@@ -431,9 +431,17 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
       return waitw(bar, parity, &own_abort, id);
     };
-    // pairs: the P and O handshakes are counted on CTA 0's barriers
+    // pairs: the P and O handshakes are counted on CTA 0's barriers.  The
+    // thread's TMEM stores or reads have completed (tcgen05 wait + fence)
+    // before it arrives; CTA 1 arrives with a CTA-scope release, since a
+    // cluster-scope release stalls the thread while the SM streams copies.
     auto arrive_lead = [&](uint32_t bar) {
-      if constexpr (PAIR) mbar_arrive_remote(mapa_shared(bar, 0)); else mbar_arrive(bar);
+      if constexpr (PAIR) {
+        if (cr == 0) mbar_arrive(bar);
+        else mbar_arrive_remote_cta(mapa_shared(bar, 0));
+      } else {
+        mbar_arrive(bar);
+      }
     };
     bool ok = true;
     int j = 0;

@@ -498,6 +498,40 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr) {
                : "memory");
 }
 
+// Arrive on an mbarrier in another CTA of the cluster, relaxed: a signal
+// that carries no data (e.g. "this CTA has finished reading a buffer").  A
+// release at cluster scope stalls the arriving thread for about a
+// microsecond while the SM streams TMA copies, so signals on the hot path
+// use this form or the CTA-scope release below.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t raddr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
+               : "memory");
+}
+
+// Arrive on an mbarrier in another CTA of the cluster with release at CTA
+// scope (orders this thread's earlier operations, which were observed
+// complete in this CTA, before the arrival).
+__device__ __forceinline__ void mbar_arrive_remote_cta(uint32_t raddr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(raddr) : "memory");
+}
+
+// Asynchronous stores into another CTA's shared memory: the bytes are
+// counted (complete_tx) on the mbarrier `rbar` of that CTA, whose waiter
+// sees the data once the phase completes.  No fence on the writing side.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(raddr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t raddr, float v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   raddr),
+               "r"(__float_as_uint(v)), "r"(rbar)
+               : "memory");
+}
+
 // try_wait with acquire at cluster scope (for phases completed by arrivals
 // or copies from the other CTA).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
