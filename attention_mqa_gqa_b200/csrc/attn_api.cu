@@ -146,6 +146,12 @@ bool shape_supported(int Sq, int d_k, int d_v) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Arrival counters of the in-kernel merge: one per (unit, head block), and
+// per CTA of the pair for the MLA kernel (each CTA merges its d rows).
+size_t merge_counters(int B, int Hkv, int head_blocks, int d_k) {
+  return (size_t)B * Hkv * head_blocks * (d_k == 576 ? 2 : 1);
+}
+
 // d = 512 prefill of groups with an even number of query heads runs on SM
 // pairs (two heads of a kv group per cluster; the K/V copies split between
 // the two SMs).
@@ -208,7 +214,8 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
   if (pl->grid_ctas > 0x7fffffffLL || (int64_t)B * Hq * Sq > 0x7fffffffLL)
     return ATTN_EUNSUPPORTED;
   const size_t n = (size_t)pl->partials * GC;
-  pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float));
+  pl->workspace_bytes = align256(n * d_v * sizeof(float)) + align256(n * sizeof(float)) +
+                        align256(merge_counters(B, Hkv, pl->head_blocks, d_k) * sizeof(unsigned int));
   return ATTN_OK;
 }
 
@@ -219,6 +226,18 @@ void set_smem(K kernel, int bytes) {
 }
 
 enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
+
+// attn_fwd's decode: decode_prepare_kernel (counters zeroed, empty
+// sequences' output written), then the split kernel with the in-kernel
+// merge, launched with programmatic stream serialization so that it starts
+// while the small kernel runs (it waits for it only before its first
+// counter update).
+template <bool BF16>
+attn_status_t launch_prepare(const attn::DecodeParams& dp, int n_counters, int d_v,
+                             cudaStream_t st) {
+  attn::decode_prepare_kernel<BF16><<<4, 256, 0, st>>>(dp, n_counters, d_v);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
 
 // The combine is launched with programmatic stream serialization: its blocks
 // may be scheduled while the split kernel finishes and wait (griddepcontrol)
@@ -268,13 +287,34 @@ attn_status_t launch_combine(const attn::DecodeParams& dp, attn::CombineParams c
 template <int DK, int DV, int NH, bool BF16>
 attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const attn::DecodeParams& dp, const attn::CombineParams& cp,
-                            const attn_plan_t& pl, cudaStream_t st, int phases) {
+                            const attn_plan_t& pl, cudaStream_t st, int phases, int n_counters) {
   using Tr = attn::DecodeTraits<DK, DV, NH>;
   static_assert(Tr::CTAS == (DK == 128 ? 2 : 1) && DK != 576, "decode_ctas_per_sm out of sync");
-  if (phases & PHASE_PARTIAL) {
-    auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
+  auto kern = attn::decode_split_kernel<DK, DV, NH, BF16>;
+  if (phases == PHASE_ALL) {  // merge in the kernel
+    if (launch_prepare<BF16>(dp, n_counters, DV, st) != ATTN_OK) return ATTN_ECUDA;
     set_smem(kern, Tr::SMEM_BYTES);
-    kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dp);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
+    cfg.blockDim = dim3(Tr::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, dp) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ECUDA;
+    }
+    return ATTN_OK;
+  }
+  if (phases & PHASE_PARTIAL) {
+    attn::DecodeParams dpp = dp;
+    dpp.counters = nullptr;  // partials only; attn_decode_combine merges them
+    set_smem(kern, Tr::SMEM_BYTES);
+    kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, dpp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   }
   if (phases & PHASE_COMBINE) return launch_combine<BF16>(dp, cp, st);
@@ -284,9 +324,13 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
 template <bool BF16>
 attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const attn::DecodeParams& dp, const attn::CombineParams& cp,
-                              const attn_plan_t& pl, cudaStream_t st, int phases) {
+                              const attn_plan_t& pl, cudaStream_t st, int phases, int n_counters) {
   using Tr = attn::MlaPairTraits;
   if (phases & PHASE_PARTIAL) {
+    const bool fused = phases == PHASE_ALL;  // merge in the kernel
+    if (fused && launch_prepare<BF16>(dp, n_counters, Tr::DV, st) != ATTN_OK) return ATTN_ECUDA;
+    attn::DecodeParams dpp = dp;
+    if (!fused) dpp.counters = nullptr;
     auto kern = attn::mla_pair_kernel<BF16>;
     set_smem(kern, Tr::SMEM_BYTES);
     cudaLaunchConfig_t cfg{};
@@ -294,17 +338,20 @@ attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, cons
     cfg.blockDim = dim3(Tr::THREADS, 1, 1);
     cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, dp) != cudaSuccess) {
+    cfg.numAttrs = fused ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, dpp) != cudaSuccess) {
       cudaGetLastError();
       return ATTN_ECUDA;
     }
+    if (fused) return ATTN_OK;
   }
   if (phases & PHASE_COMBINE) return launch_combine<BF16>(dp, cp, st);
   return ATTN_OK;
@@ -418,6 +465,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     dp.head_blocks = pl.head_blocks;
     dp.scale_log2 = scale_log2;
     dp.timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);
+    const int n_counters = (int)merge_counters(B, Hkv, pl.head_blocks, d_k);
+    dp.counters = reinterpret_cast<unsigned int*>(
+        reinterpret_cast<uint8_t*>(workspace) + align256(n * d_v * sizeof(float)) +
+        align256(n * sizeof(float)));
+    dp.out = out;
+    dp.o_sb = so.b;
+    dp.o_sh = so.h;
+    dp.o_ss = so.s;
+    dp.lse = lse;
     attn::CombineParams cp{};
     cp.ws_o = dp.ws_o;
     cp.ws_lse = dp.ws_lse;
@@ -436,13 +492,13 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     cp.ranges = pl.kv_ranges;
     cp.tile_shift = decode_pairs(d_k) ? attn::MlaPairTraits::TILE_SHIFT : 7;
     if (d_k == 128)
-      return bf16 ? launch_decode<128, 128, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
-                  : launch_decode<128, 128, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
+      return bf16 ? launch_decode<128, 128, 16, true>(mq, mk, mv, dp, cp, pl, st, phases, n_counters)
+                  : launch_decode<128, 128, 16, false>(mq, mk, mv, dp, cp, pl, st, phases, n_counters);
     if (d_k == 512)
-      return bf16 ? launch_decode<512, 512, 16, true>(mq, mk, mv, dp, cp, pl, st, phases)
-                  : launch_decode<512, 512, 16, false>(mq, mk, mv, dp, cp, pl, st, phases);
-    return bf16 ? launch_mla_pair<true>(mq, mk, mv, dp, cp, pl, st, phases)
-                : launch_mla_pair<false>(mq, mk, mv, dp, cp, pl, st, phases);
+      return bf16 ? launch_decode<512, 512, 16, true>(mq, mk, mv, dp, cp, pl, st, phases, n_counters)
+                  : launch_decode<512, 512, 16, false>(mq, mk, mv, dp, cp, pl, st, phases, n_counters);
+    return bf16 ? launch_mla_pair<true>(mq, mk, mv, dp, cp, pl, st, phases, n_counters)
+                : launch_mla_pair<false>(mq, mk, mv, dp, cp, pl, st, phases, n_counters);
   }
 
   const bool pairs = prefill_pairs(d_k, G);

@@ -27,26 +27,6 @@ struct CombineParams {
   int col_chunks;  // blocks per unit = ceil(G * Sq / cols)
 };
 
-// Largest range index r with floor(r * T / R) <= x (the range holding tile x).
-__device__ __forceinline__ long long range_of(long long x, long long T, long long R) {
-  return ((x + 1) * R + T - 1) / T - 1;
-}
-
-// (m, l) <- the log-sum-exp statistics of the union of two sets: maximum m
-// and sum of exp(x - m).  Symmetric in its two operands (bit for bit), so
-// both lanes of a butterfly exchange end with the same value.
-__device__ __forceinline__ void merge_stat(float& m, float& l, float m2, float l2) {
-  if (m2 == -INFINITY) return;
-  if (m == -INFINITY) {
-    m = m2;
-    l = l2;
-    return;
-  }
-  const float M = fmaxf(m, m2);
-  l = l * __expf(m - M) + l2 * __expf(m2 - M);
-  m = M;
-}
-
 constexpr int kCombineThreads = 128;
 
 // One block per (unit u = (b, kv head), chunk of `cols` columns).  The

@@ -54,6 +54,15 @@ struct DecodeParams {
   int ranges, head_blocks;
   float scale_log2;      // scale * log2(e)
   uint64_t timeout_ns;
+  // In-kernel merge (attn_fwd): the last CTA to finish a piece of a unit
+  // merges the unit's pieces into `out` / `lse`.  `counters` (one per unit
+  // and head block, per CTA of a pair for the MLA kernel) are zeroed by
+  // decode_prepare_kernel just before.  counters == nullptr leaves the merge
+  // to combine_kernel (attn_decode_partial, then attn_decode_combine).
+  unsigned int* counters;
+  void* out;                  // [B, Hq, Sq, d_v]
+  int64_t o_sb, o_sh, o_ss;   // element strides of out
+  float* lse;                 // [B, Hq, Sq] or NULL
 };
 
 constexpr uint32_t ceil_pow2_cols(uint32_t n) {
@@ -105,11 +114,13 @@ struct DecodeTraits {
   static constexpr int OFF_L = OFF_ALPHA + NH * 4;              // float [NH] final sums
   static constexpr int OFF_SCAN = OFF_L + NH * 4;               // int64 [8] block scan
   static constexpr int OFF_SCHED = OFF_SCAN + 64;               // int [4] range start
-  static constexpr int OFF_FLAGS = OFF_SCHED + 16;              // int [4]: any[2], abort, tmem
-  static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
+  static constexpr int OFF_POS = OFF_SCHED + 16;                // int64 [4] range position
+  static constexpr int OFF_FLAGS = OFF_POS + 32;                // int [4]: any[2], abort, tmem
+  static constexpr int OFF_MERGE = OFF_FLAGS + 16;              // int: this CTA merges a unit
+  static constexpr int OFF_BAR = (OFF_MERGE + 16 + 7) & ~7;
   // full[RING_G], empty[RING_G], s_full[2], s_free[2], p_full[NPT], o_done[NPT], q_full[NQ],
   // q_free[NQ], red_full[2], stat_ready[2], drain
-  static constexpr int NBAR = 2 * RING_G + 9 + 2 * NPT + 2 * NQ;
+  static constexpr int NBAR = 2 * RING_G + 11 + 2 * NPT + 2 * NQ;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;  // + alignment slack
   static constexpr int TMEM_S = 0;                  // S^T double buffer: 2 x NH columns
   static constexpr int TMEM_O = 2 * NH;             // O^T: DVB x NH columns
@@ -161,8 +172,13 @@ struct PieceWalker {
   const int32_t* skv;
   int B, Hkv, shift;
   int b, kvh, off, remaining;
+  long long gpos = 0;  // global index (over all units' tiles) of the next piece's first tile
 
   __device__ bool next(int& pb, int& pkvh, int& tile0, int& ntiles) {
+    long long g;
+    return next(pb, pkvh, tile0, ntiles, g);
+  }
+  __device__ bool next(int& pb, int& pkvh, int& tile0, int& ntiles, long long& gstart) {
     if (remaining <= 0) return false;
     const int tb = key_tiles(skv[b], shift);
     const int n = min(remaining, tb - off);
@@ -170,6 +186,8 @@ struct PieceWalker {
     pkvh = kvh;
     tile0 = off;
     ntiles = n;
+    gstart = gpos;
+    gpos += n;
     remaining -= n;
     off = 0;
     if (remaining > 0) {
@@ -185,9 +203,10 @@ struct PieceWalker {
 // Range `r` of min(R, T) equal ranges over the T concatenated key tiles of
 // all units (unit u = b * Hkv + kvh holds ceil(skv[b] / 128) tiles).  Called
 // by all threads of the CTA; leaves the range's first unit, tile offset and
-// length in sched[0..3] (length 0: no range r).
+// length in sched[0..3] (length 0: no range r), and in pos[0..2] the range's
+// first global tile, T and the number of ranges in use.
 __device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv, int shift, int R,
-                                             int r, long long* scan, int* sched) {
+                                             int r, long long* scan, int* sched, long long* pos) {
   const int tid = threadIdx.x;
   const int nt = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -214,7 +233,12 @@ __device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv,
   const long long Re = T < R ? T : R;
   const long long x0 = r < Re ? (long long)r * T / Re : T;
   const long long x1 = r < Re ? (long long)(r + 1) * T / Re : T;
-  if (tid == 0) sched[3] = (int)(x1 - x0);
+  if (tid == 0) {
+    sched[3] = (int)(x1 - x0);
+    pos[0] = x0;
+    pos[1] = T;
+    pos[2] = Re;
+  }
   long long run = before + v - mine;  // tiles of sequences before `lo`
   for (int b = lo; b < hi; ++b) {
     const int tb = key_tiles(skv[b], shift);
@@ -227,6 +251,174 @@ __device__ __forceinline__ void locate_range(const int32_t* skv, int B, int Hkv,
     run += tb;
   }
   __syncthreads();
+}
+
+// Largest range index r with floor(r * T / R) <= x (the range holding tile x).
+__device__ __forceinline__ long long range_of(long long x, long long T, long long R) {
+  return ((x + 1) * R + T - 1) / T - 1;
+}
+
+// (m, l) <- the log-sum-exp statistics of the union of two sets: maximum m
+// and sum of exp(x - m).  Symmetric in its two operands (bit for bit), so
+// both lanes of a butterfly exchange end with the same value.
+__device__ __forceinline__ void merge_stat(float& m, float& l, float m2, float l2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2;
+    l = l2;
+    return;
+  }
+  const float M = fmaxf(m, m2);
+  l = l * __expf(m - M) + l2 * __expf(m2 - M);
+  m = M;
+}
+
+// Arrival on a unit's counter after this CTA wrote its piece of the unit
+// (ntiles of the unit's tb key tiles).  Called by every thread of the
+// softmax warps (each warp converged) after its partial-output stores; the
+// warps meet on two mbarriers with bounded waits (done: every warp's stores
+// issued; flag: the leader warp's verdict), phase `parity`.  One thread
+// updates the counter with an acquire-release atomic at GPU scope, whose
+// release covers the CTA's stores (they precede it through the `done`
+// barrier) and whose acquire, in the CTA that completes the unit, makes
+// every other piece visible to the merge that follows.  Returns in every
+// caller whether this CTA completed the unit.  The counters were zeroed by
+// the kernel before this one in the stream; griddepcontrol.wait waits for it.
+__device__ __forceinline__ bool arrive_last(unsigned int* counter, int ntiles, int tb,
+                                            uint32_t bar_done, uint32_t bar_flag,
+                                            uint32_t parity, bool leader, volatile int* flag,
+                                            volatile int* abort, uint64_t timeout_ns) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_done);
+  if (leader) {
+    const bool ok = mbar_wait_warp(bar_done, parity, abort, timeout_ns, 19);
+    if (lane == 0) {
+      int last = 0;
+      if (ok) {
+        pdl_wait();
+        unsigned int old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                     : "=r"(old)
+                     : "l"(counter), "r"((unsigned int)ntiles)
+                     : "memory");
+        last = old + (unsigned int)ntiles == (unsigned int)tb;
+      }
+      *flag = last;
+      mbar_arrive(bar_flag);
+    }
+    __syncwarp();
+  }
+  return mbar_wait_warp(bar_flag, parity, abort, timeout_ns, 20) && *flag != 0;
+}
+
+// Merge of the pieces s = 0 .. n-1 of one unit (workspace slots slot0 + s)
+// for columns [c0, c0 + ncol) of the unit's GC and d_v elements [d0, d0 +
+// 4 * F4 * TPC) of each: out = sum_s exp(lse_s - L) o_s, L = log sum_s
+// exp(lse_s), adding the pieces in range order (bitwise reproducible
+// whichever CTA merges).  A group of TPC adjacent lanes per column (TPC a
+// power of two <= 32), F4 float4 per thread; t in [0, TPC * ncol) -- other
+// threads return.  L: each lane of the group folds every TPC-th piece, then
+// a butterfly of symmetric merges gives every lane the same L; the
+// weighted sum then takes PP pieces per round with all their loads in
+// flight.  With write_lse, L goes to the output LSE.  Loads bypass L1: the
+// pieces were written by other SMs.
+template <bool BF16, int TPC, int F4>
+__device__ __forceinline__ void merge_unit(const DecodeParams& p, int DV, int GC, long long slot0,
+                                           int n, int b, int kvh, int c0, int ncol, int d0,
+                                           bool write_lse, int t) {
+  constexpr int PP = F4 >= 16 ? 1 : 16 / F4;  // pieces per round: <= 16 float4 loads in flight
+  const int cc = t / TPC, j = t % TPC;
+  if (cc >= ncol) return;  // whole groups leave together
+  const int lane = threadIdx.x & 31;
+  const unsigned int gmask = (TPC >= 32) ? 0xffffffffu
+                                         : (((1u << TPC) - 1u) << (lane & ~(TPC - 1) & 31));
+  const int col = c0 + cc;
+  const float* lse_c = p.ws_lse + slot0 * GC + col;
+  float m = -INFINITY, l = 0.f;
+  for (int s = j; s < n; s += TPC) merge_stat(m, l, __ldcg(lse_c + (long long)s * GC), 1.f);
+#pragma unroll
+  for (int o = TPC / 2; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(gmask, m, o);
+    const float l2 = __shfl_xor_sync(gmask, l, o);
+    merge_stat(m, l, m2, l2);
+  }
+  const float L = (m == -INFINITY || !(l > 0.f)) ? -INFINITY : m + __logf(l);
+  float4 acc[F4];
+#pragma unroll
+  for (int k = 0; k < F4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (L != -INFINITY) {
+    const float4* o_c = reinterpret_cast<const float4*>(p.ws_o + (slot0 * GC + col) * (long long)DV + d0);
+    const long long piece_f4 = (long long)GC * DV / 4;
+    for (int s = 0; s < n; s += PP) {
+      float w[PP];
+      float4 v[PP][F4];
+#pragma unroll
+      for (int q = 0; q < PP; ++q) {
+        const bool in = s + q < n;
+        w[q] = in ? __ldcg(lse_c + (long long)(s + q) * GC) : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < F4; ++k)
+          v[q][k] = in ? __ldcg(o_c + (s + q) * piece_f4 + j + k * TPC) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < PP; ++q) {  // pieces in range order
+        const float wq = s + q < n ? __expf(w[q] - L) : 0.f;
+#pragma unroll
+        for (int k = 0; k < F4; ++k) {
+          acc[k].x = fmaf(wq, v[q][k].x, acc[k].x);
+          acc[k].y = fmaf(wq, v[q][k].y, acc[k].y);
+          acc[k].z = fmaf(wq, v[q][k].z, acc[k].z);
+          acc[k].w = fmaf(wq, v[q][k].w, acc[k].w);
+        }
+      }
+    }
+  }
+  const int h = kvh * p.G + col / p.Sq, qi = col % p.Sq;
+  uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
+                  ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)qi * p.o_ss + d0) * 2;
+#pragma unroll
+  for (int k = 0; k < F4; ++k)
+    *reinterpret_cast<uint2*>(orow + (j + k * TPC) * 8) =
+        make_uint2(pack2(acc[k].x, acc[k].y, BF16), pack2(acc[k].z, acc[k].w, BF16));
+  if (write_lse && j == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.Sq + qi] = L;
+}
+
+// The merge of (b, kv head) pieces, located from one of them: the piece
+// starting at global tile gstart, tile0 tiles into its unit of tb tiles.
+// Returns the first workspace slot and the number of pieces.
+__device__ __forceinline__ int unit_pieces(long long gstart, int tile0, int tb, int unit,
+                                           const long long* pos, long long& slot0) {
+  const long long su = gstart - tile0;  // the unit's first global tile
+  const long long r_lo = range_of(su, pos[1], pos[2]);
+  slot0 = r_lo + unit;
+  return (int)(range_of(su + tb - 1, pos[1], pos[2]) - r_lo + 1);
+}
+
+// Zeroes the arrival counters of the in-kernel merge and writes the output
+// of sequences with no key (out = 0, LSE = -inf): no piece covers them.
+// Lets the decode kernel, launched after it with programmatic stream
+// serialization, start at once; that kernel waits for this one to finish
+// only before its first counter update.
+template <bool BF16>
+__global__ void __launch_bounds__(256) decode_prepare_kernel(const DecodeParams p, int n_counters,
+                                                             int DV) {
+  pdl_launch_dependents();
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nth = gridDim.x * blockDim.x;
+  for (int i = tid; i < n_counters; i += nth) p.counters[i] = 0;
+  const int rows = p.Hq * p.Sq;
+  for (int b = 0; b < p.B; ++b) {
+    if (p.skv[b] != 0) continue;
+    for (int i = tid; i < rows * (DV / 8); i += nth) {
+      const int row = i / (DV / 8), c8 = i % (DV / 8);
+      const int h = row / p.Sq, qi = row % p.Sq;
+      *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) +
+                                ((int64_t)b * p.o_sb + (int64_t)h * p.o_sh + (int64_t)qi * p.o_ss +
+                                 c8 * 8) * 2) = make_uint4(0u, 0u, 0u, 0u);
+      if (c8 == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.Sq + qi] = -INFINITY;
+    }
+  }
 }
 
 template <int DK, int DV, int NH, bool BF16>
@@ -256,6 +448,8 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
   float* l_sm = reinterpret_cast<float*>(smem + T::OFF_L);
   long long* scan = reinterpret_cast<long long*>(smem + T::OFF_SCAN);
   int* sched = reinterpret_cast<int*>(smem + T::OFF_SCHED);
+  long long* pos = reinterpret_cast<long long*>(smem + T::OFF_POS);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + T::OFF_MERGE);
   volatile int* flags = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
   volatile int* abort_flag = flags + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 12);
@@ -271,6 +465,8 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
   const uint32_t red_full = q_free + 8 * T::NQ;           // [2]
   const uint32_t stat_ready = red_full + 16;              // [2]
   const uint32_t drain = stat_ready + 16;
+  const uint32_t mg_done = drain + 8;     // in-kernel merge: the softmax warps' stores fenced
+  const uint32_t mg_flag = mg_done + 8;   // in-kernel merge: this CTA completed the unit
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -295,6 +491,8 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       mbar_init(q_free + 8 * i, 1);
     }
     mbar_init(drain, 1);
+    mbar_init(mg_done, T::SOFTMAX_THREADS / 32);
+    mbar_init(mg_flag, 1);
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
@@ -305,7 +503,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
     tmem_relinquish();
   }
   if (threadIdx.x == 0) pdl_launch_dependents();  // the combine may be scheduled now
-  locate_range(p.skv, p.B, p.Hkv, 7, p.ranges, rng, scan, sched);  // contains __syncthreads
+  locate_range(p.skv, p.B, p.Hkv, 7, p.ranges, rng, scan, sched, pos);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -321,6 +519,7 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
     w.kvh = sched[1];
     w.off = sched[2];
     w.remaining = count;
+    w.gpos = pos[0];
     return w;
   };
 
@@ -508,9 +707,10 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
       named_bar_sync(1, T::SOFTMAX_THREADS);
 
       PieceWalker w = walker();
-      int b, kvh, t0, n, j = 0, r = 0;
+      int b, kvh, t0, n, j = 0, r = 0, pc = 0;
+      long long gstart;
       bool ok = true;
-      while (ok && w.next(b, kvh, t0, n)) {
+      while (ok && w.next(b, kvh, t0, n, gstart)) {
         const int skv_b = p.skv[b];
         const int64_t slot_id = (int64_t)rng + (int64_t)b * p.Hkv + kvh;  // workspace slot
         float l[HH];
@@ -692,6 +892,23 @@ __global__ void __launch_bounds__(DecodeTraits<DK, DV, NH>::THREADS, DecodeTrait
             }
           }
           tc_fence_before();
+          // the CTA that completes the unit's (head block's) key tiles merges
+          // the unit's pieces into the output
+          if (p.counters) {
+            const int unit = b * p.Hkv + kvh;
+            const int tb = key_tiles(skv_b, 7);
+            const bool last = arrive_last(p.counters + (int64_t)unit * p.head_blocks + hb, n, tb,
+                                          mg_done, mg_flag, pc & 1, warp == 2, merge_flag,
+                                          &own_abort, p.timeout_ns);
+            ++pc;
+            if (last) {
+              long long slot0;
+              const int np = unit_pieces(gstart, t0, tb, unit, pos, slot0);
+              constexpr int TPC = T::SOFTMAX_THREADS / NH;  // threads per column
+              merge_unit<BF16, TPC, DV / 4 / TPC>(p, DV, GC, slot0, np, b, kvh, hb * NH, nvalid,
+                                                  0, true, st);
+            }
+          }
         }
       }
       if (!ok) *abort_flag = 1;

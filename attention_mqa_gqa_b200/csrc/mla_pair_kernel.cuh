@@ -73,11 +73,13 @@ struct MlaPairTraits {
   static constexpr int OFF_LPEER = OFF_L + NH * 4;          // float [NH] peer sums
   static constexpr int OFF_SCAN = OFF_LPEER + NH * 4;       // int64 [8]
   static constexpr int OFF_SCHED = OFF_SCAN + 64;           // int [4]
-  static constexpr int OFF_FLAGS = OFF_SCHED + 16;          // int [4]: any[2], abort, tmem
-  static constexpr int OFF_BAR = (OFF_FLAGS + 16 + 7) & ~7;
+  static constexpr int OFF_POS = OFF_SCHED + 16;            // int64 [4] range position
+  static constexpr int OFF_FLAGS = OFF_POS + 32;            // int [4]: any[2], abort, tmem
+  static constexpr int OFF_MERGE = OFF_FLAGS + 16;          // int: this CTA merges a unit half
+  static constexpr int OFF_BAR = (OFF_MERGE + 16 + 7) & ~7;
   // full[3] empty[3] q_full q_free s_full[2] s_free[2] p_local p_recv p_peer o_done
-  // red_full[2] stat_ready[2] xmax_full[2] lsum_full drain
-  static constexpr int NBAR = 2 * RING_G + 2 + 2 + 2 + 3 + 1 + 2 + 2 + 2 + 1 + 1;
+  // red_full[2] stat_ready[2] xmax_full[2] lsum_full drain mg_done mg_flag
+  static constexpr int NBAR = 2 * RING_G + 2 + 2 + 2 + 3 + 1 + 2 + 2 + 2 + 1 + 1 + 2;
   static constexpr int PT_PEER_BYTES = TILE * NHC * 2;     // P^T rows one CTA sends the other
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int SOFTMAX_THREADS = 256;
@@ -135,6 +137,8 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
   float* lpeer = reinterpret_cast<float*>(smem + T::OFF_LPEER);
   long long* scan = reinterpret_cast<long long*>(smem + T::OFF_SCAN);
   int* sched = reinterpret_cast<int*>(smem + T::OFF_SCHED);
+  long long* pos = reinterpret_cast<long long*>(smem + T::OFF_POS);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + T::OFF_MERGE);
   volatile int* flags = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
   volatile int* abort_flag = flags + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 12);
@@ -154,6 +158,8 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
   const uint32_t xmax_full = stat_ready + 16;  // [2] peer maxima landed
   const uint32_t lsum_full = xmax_full + 16;   // peer sums landed
   const uint32_t drain = lsum_full + 8;
+  const uint32_t mg_done = drain + 8;     // in-kernel merge: the softmax warps' stores fenced
+  const uint32_t mg_flag = mg_done + 8;   // in-kernel merge: this CTA completed its unit half
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -179,6 +185,8 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
     mbar_init(o_done, 1);
     mbar_init(lsum_full, 1);
     mbar_init(drain, 1);
+    mbar_init(mg_done, T::SOFTMAX_THREADS / 32);
+    mbar_init(mg_flag, 1);
     flags[0] = 0;
     flags[1] = 0;
     flags[2] = 0;
@@ -192,7 +200,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
     tmem_relinquish_pair();
   }
   if (threadIdx.x == 0) pdl_launch_dependents();  // the combine may be scheduled now
-  locate_range(p.skv, p.B, p.Hkv, T::TILE_SHIFT, p.ranges, rng, scan, sched);
+  locate_range(p.skv, p.B, p.Hkv, T::TILE_SHIFT, p.ranges, rng, scan, sched, pos);
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers and the pair's TMEM exist
   tc_fence_after();
@@ -208,6 +216,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
     w.kvh = sched[1];
     w.off = sched[2];
     w.remaining = count;
+    w.gpos = pos[0];
     return w;
   };
 
@@ -431,8 +440,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
 
       PieceWalker w = walker();
       int b, kvh, t0, n, j = 0, r = 0, pc = 0;
+      long long gstart;
       bool ok = true;
-      while (ok && w.next(b, kvh, t0, n)) {
+      while (ok && w.next(b, kvh, t0, n, gstart)) {
         const int skv_b = p.skv[b];
         const int64_t slot_id = (int64_t)rng + (int64_t)b * p.Hkv + kvh;
         float l[HH];
@@ -610,7 +620,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
               // the same sum in both CTAs: CTA 0's keys first
               const float L = cr == 0 ? own + lpeer[st] : lpeer[st] + own;
               l_sm[st] = L;
-              if (cr == 0 && st < nvalid)
+              // both CTAs write the (identical) LSE: the merge of either
+              // half of the output reads it
+              if (st < nvalid)
                 p.ws_lse[slot_id * p.G + hb * NH + st] =
                     L > 0.f ? (m_sm[st] + __log2f(L)) * 0.69314718055994531f : -INFINITY;
               m_sm[st] = -INFINITY;  // the next piece starts afresh
@@ -642,6 +654,24 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
             }
           }
           tc_fence_before();
+          // the CTA that completes its half (d rows) of the unit's key tiles
+          // merges that half of the unit's pieces into the output
+          if (p.counters) {
+            const int unit = b * p.Hkv + kvh;
+            const int tb = key_tiles(skv_b, T::TILE_SHIFT);
+            const bool last = arrive_last(
+                p.counters + ((int64_t)unit * p.head_blocks + hb) * 2 + cr, n, tb, mg_done,
+                mg_flag, (pc - 1) & 1, warp == 2, merge_flag, &own_abort, p.timeout_ns);
+            if (last) {
+              long long slot0;
+              const int np = unit_pieces(gstart, t0, tb, unit, pos, slot0);
+              constexpr int TPC = T::SOFTMAX_THREADS / NH;  // threads per head
+              for (int m = 0; m < 2; ++m)  // d rows 256 m + 128 cr .. + 127
+                merge_unit<BF16, TPC, 128 / 4 / TPC>(p, T::DV, p.G, slot0, np, b, kvh, hb * NH,
+                                                     nvalid, 256 * m + 128 * (int)cr,
+                                                     cr == 0 && m == 0, st);
+            }
+          }
         }
       }
       if (!ok) *abort_flag = 1;

@@ -5,7 +5,8 @@
 
 Default workload: MQA decode at head_dim 512 (B=32, Hq=16, Hkv=1, per-sequence
 KV length uniform in [1024, 8192], bf16): one step = one decode forward of
-the whole batch (split-KV partial kernel + LSE combine).  The metric is the
+the whole batch (split-KV kernel, whose last CTA per sequence merges the
+pieces, after a small kernel that zeroes its arrival counters).  The metric is the
 KV-cache bytes read per second (each cached K/V byte counted once).  The
 same line carries, measured in the same run and each in an object of its
 own: the d=512 MQA causal prefill (B=2, Hq=16, S=4096; key "prefill"),
@@ -290,10 +291,14 @@ class GpuRunner:
                            self.stream)
 
     def call(self, entry="attn_fwd"):
+        """One launch group: "attn_fwd" (a whole step; for top-k, the row
+        gather first), "forward" (attn_fwd without the gather), "gather"."""
         if entry == "gather":
             return self.gather()
         if self.topk and entry == "attn_fwd":
             self.gather()
+        if entry == "forward":
+            entry = "attn_fwd"
         rc = self.b.fwd_raw(*self.args(), entry=entry)
         if rc != 0:
             raise self.b.AttnError(rc, entry)
@@ -346,10 +351,11 @@ class GpuRunner:
         (captured two steps at a time); CUDA events on the replay stream.
         Returns (total_ms, dominant kernel mean ms, other kernel mean ms).
         The dominant kernel's duration is timed the same way over graphs of
-        20 back-to-back launches of that kernel alone (for decode the split
-        kernel, whose inputs do not depend on the combine); the combine's is
-        the step time minus that (and minus the row gather of a top-k step,
-        timed the same way, in ``self.gather_ms``)."""
+        20 back-to-back launches of it alone: for decode, attn_fwd's split
+        kernel with the merge of the pieces inside it (with the few-
+        microsecond kernel that zeroes its arrival counters and lets it start
+        early); for a top-k step the row gather is timed on its own too (in
+        ``self.gather_ms``), the rest of the step being the other time."""
         per = steps_per_graph(steps)
         graph, side = self._graph(per)
         reps = []
@@ -358,7 +364,7 @@ class GpuRunner:
         del graph
         if not self.decode:
             return total, total / steps, 0.0
-        kg, kside = self._graph(20, "attn_decode_partial")
+        kg, kside = self._graph(20, "forward")
         k_ms = self._replay_ms(kg, kside, 10, 1) / 200
         del kg
         self.gather_ms = 0.0
@@ -630,7 +636,12 @@ def dominant_roofline(w, g, keys, k_ms, other_ms, total_ms, peaks, peak_src):
     roof["kernel"] = kname
     roof["kernel_ms"] = round(k_ms, 5)
     if g.decode:
-        roof["combine_ms"] = round(other_ms, 5)
+        # the pieces of each (sequence, kv head) are merged inside the split
+        # kernel by the CTA that finishes the unit; kernel_ms covers the
+        # launch with its small counter-zeroing kernel (launched just before
+        # it, overlapping its start)
+        roof["merge"] = "in kernel (last CTA of a unit)"
+        roof["other_ms"] = round(other_ms, 5)
     return roof
 
 

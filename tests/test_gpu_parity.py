@@ -1,8 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Small cases and the full-size decode workloads compare every output
-element; the full-size prefill workloads compare sampled rows (the oracle
-evaluates those rows one by one).  Tolerance:
+Small cases and the full-size workloads compare every output element and
+LSE.  Tolerance:
 |gpu - oracle| <= 1e-2 + 1e-2*|oracle| per element, |dLSE| <= 1e-3.
 """
 import math
@@ -93,6 +92,42 @@ def test_decode_fp16():
 
 def test_decode_zero_length_sequence():
     _case(3, 16, 1, 1, [0, 300, 0], 512, 512, seed=5, max_skv=300)
+
+
+@pytest.mark.parametrize("case", ["mqa_d512", "gqa_extend", "mla"])
+def test_decode_two_phase_entry_points(case):
+    """attn_decode_partial followed by attn_decode_combine (the separate
+    merge kernel) gives the attention too; attn_fwd merges inside the split
+    kernel instead."""
+    from attention_mqa_gqa_b200 import binding
+
+    if case == "mqa_d512":
+        w, inp = wl.make_case(3, 16, 1, 1, [2000, 0, 777], 512, 512, seed=71)
+    elif case == "gqa_extend":
+        w, inp = wl.make_case(2, 16, 2, 4, [300, 3], 128, 128, seed=72)
+    else:
+        w, inp = wl.make_case(2, 128, 1, 1, [3000, 300], 576, 512, mla=True, seed=73,
+                              scale=192 ** -0.5)
+    dev = to_device(inp)
+    q, k, v = dev["q"], dev["k"], dev["v"]
+    B, Hq, Sq, dk = q.shape
+    out = torch.full((B, Hq, Sq, v.shape[-1]), float("nan"), dtype=q.dtype, device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), dtype=torch.float32, device="cuda")
+    n = binding.workspace_bytes(B, Hq, k.shape[1], Sq, dev["max_skv"], dk, v.shape[-1])
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    st = lambda t: binding.Strides(t.stride(0), t.stride(1), t.stride(2))
+    for entry in ("attn_decode_partial", "attn_decode_combine"):
+        rc = binding.fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, Hq, k.shape[1], Sq, dev["skv"].data_ptr(),
+                             dev["max_skv"], dk, v.shape[-1], w.scale, w.causal,
+                             binding.dtype_code(q.dtype), st(q), st(k), st(v), st(out),
+                             ws.data_ptr(), n, torch.cuda.current_stream().cuda_stream,
+                             entry=entry)
+        assert rc == binding.ATTN_OK
+    torch.cuda.synchronize()
+    assert binding.last_device_error() == binding.ATTN_OK
+    ref_o, ref_l = oracle_full(w, inp)
+    compare(out, lse, ref_o, ref_l, f"two-phase {case}")
 
 
 def test_decode_strided_views():

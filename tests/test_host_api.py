@@ -64,7 +64,10 @@ def test_plan_decode_invariants(lib):
         assert pl["partials"] == pl["kv_ranges"] + B * Hkv
         n = pl["partials"] * G
         r256 = lambda x: (x + 255) // 256 * 256
-        assert pl["workspace_bytes"] == r256(n * dv * 4) + r256(n * 4)
+        # partial outputs, partial LSEs, then the in-kernel merge's arrival
+        # counters: one per (unit, head block), per CTA of the pair for MLA
+        counters = B * Hkv * pl["head_blocks"] * (2 if dk == 576 else 1)
+        assert pl["workspace_bytes"] == r256(n * dv * 4) + r256(n * 4) + r256(counters * 4)
 
 
 def _ranges_pieces(skv, Hkv, R):
@@ -129,7 +132,8 @@ def test_plan_extend_takes_decode_path(lib):
         assert pl["head_blocks"] == -(-G * Sq // 16)
         n = pl["partials"] * G * Sq
         r256 = lambda x: (x + 255) // 256 * 256
-        assert pl["workspace_bytes"] == r256(n * dk * 4) + r256(n * 4)
+        counters = 5 * Hkv * pl["head_blocks"]
+        assert pl["workspace_bytes"] == r256(n * dk * 4) + r256(n * 4) + r256(counters * 4)
     for Sq in (3, 32, 100):  # not a power of two, or too many columns
         assert binding.plan(5, 64, 8, Sq, 4096, 128, 128, num_sms=148)["path"] == 0
     assert binding.plan(5, 128, 128, 4, 4096, 192, 128, num_sms=148)["path"] == 0
