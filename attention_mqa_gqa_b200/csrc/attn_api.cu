@@ -20,6 +20,7 @@
 #include "gather_rows.cuh"
 #include "mla_pair_kernel.cuh"
 #include "prefill_kernel.cuh"
+#include "prefill_ab_kernel.cuh"
 
 namespace {
 
@@ -152,10 +153,10 @@ size_t merge_counters(int B, int Hkv, int head_blocks, int d_k) {
   return (size_t)B * Hkv * head_blocks * (d_k == 576 ? 2 : 1);
 }
 
-// d = 512 prefill of groups with an even number of query heads runs on SM
-// pairs (two heads of a kv group per cluster; the K/V copies split between
-// the two SMs).
-bool prefill_pairs(int d_k, int G) { return d_k == 512 && G % 2 == 0; }
+// d = 512 prefill runs on SM pairs that split the two matmuls: one CTA
+// computes S and the softmax, the other holds O and runs PV (one work item
+// = 128 query rows of one head per pair).
+bool prefill_split_matmuls(int d_k) { return d_k == 512; }
 
 // Columns (head x query) per decode CTA for d_k in {128, 512}.
 constexpr int kDecodeCols = 16;
@@ -183,13 +184,13 @@ attn_status_t plan_impl(int B, int Hq, int Hkv, int Sq, int max_skv, int d_k, in
   const int G = Hq / Hkv;
   if (!decode_path(Sq, d_k)) {
     pl->path = 0;
-    pl->dv_parts = d_v / (d_v >= 512 ? 256 : 128);
+    pl->dv_parts = prefill_split_matmuls(d_k) ? 1 : d_v / 128;
     const int64_t n_qt = (Sq + 127) / 128;
     const int64_t items = n_qt * Hq * (int64_t)B * pl->dv_parts;  // persistent CTAs walk these
     if (items > 0x7fffffffLL) return ATTN_EUNSUPPORTED;
-    if (prefill_pairs(d_k, G)) {  // clusters of two CTAs, one item per pair of heads
-      const int64_t units = items / 2, pairs = num_sms / 2;
-      pl->grid_ctas = 2 * (units < pairs ? units : pairs);
+    if (prefill_split_matmuls(d_k)) {  // clusters of two CTAs, one item per pair
+      const int64_t pairs = num_sms / 2;
+      pl->grid_ctas = 2 * (items < pairs ? items : pairs);
     } else {
       pl->grid_ctas = items < num_sms ? items : num_sms;
     }
@@ -388,6 +389,32 @@ attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const
   return ATTN_OK;
 }
 
+template <bool BF16>
+attn_status_t launch_prefill_ab(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                const attn::PrefillParams& pp, const attn_plan_t& pl,
+                                cudaStream_t st) {
+  using Tr = attn::PrefillABTraits;
+  auto kern = attn::prefill_ab_kernel<BF16>;
+  set_smem(kern, Tr::SMEM_BYTES);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
+  cfg.blockDim = dim3(Tr::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ECUDA;
+  }
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -501,14 +528,17 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
                 : launch_mla_pair<false>(mq, mk, mv, dp, cp, pl, st, phases, n_counters);
   }
 
-  const bool pairs = prefill_pairs(d_k, G);
-  // pairs: each CTA copies 64 of a K tile's 128 keys (four chunks per copy)
-  if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, pairs ? 4 : 2,
-                      pairs ? 64 : 128))
+  const bool split = prefill_split_matmuls(d_k);
+  // split matmuls: Q and K copies of 4 chunks x 128 rows, V copies of 8
+  // chunks x 64 keys (64 KB each); otherwise 2 chunks x 128 rows
+  if (!make_chunk_map(&mk, k, dtype, d_k, max_skv, Hkv, B, sk.s, sk.h, sk.b, split ? 4 : 2))
     return ATTN_ECUDA;
-  if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, 2)) return ATTN_ECUDA;
+  if (!make_chunk_map(&mv, v, dtype, d_v, max_skv, Hkv, B, sv.s, sv.h, sv.b, split ? 8 : 2,
+                      split ? 64 : 128))
+    return ATTN_ECUDA;
   CUtensorMap mq;
-  if (!make_chunk_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b, 2)) return ATTN_ECUDA;
+  if (!make_chunk_map(&mq, q, dtype, d_k, Sq, Hq, B, sq.s, sq.h, sq.b, split ? 4 : 2))
+    return ATTN_ECUDA;
   attn::PrefillParams pp{};
   pp.out = out;
   pp.o_sb = so.b;
@@ -523,8 +553,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.Sq = Sq;
   pp.n_qtiles = (Sq + 127) / 128;
   pp.dv_parts = pl.dv_parts;
-  pp.pairs = pairs ? 1 : 0;
-  pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts / (pairs ? 2 : 1);  // per CTA or per pair
+  pp.pairs = 0;
+  pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;  // per CTA, or per pair (split matmuls)
   {
     // K/V bytes of one kv head over the batch; blocks of kv heads whose
     // K/V stays within ~40 MB of the 126 MB L2
@@ -543,11 +573,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   if (d_k == 192)
     return bf16 ? launch_prefill<192, 128, true>(mq, mk, mv, pp, pl, st)
                 : launch_prefill<192, 128, false>(mq, mk, mv, pp, pl, st);
-  if (pairs)
-    return bf16 ? launch_prefill<512, 256, true, true>(mq, mk, mv, pp, pl, st)
-                : launch_prefill<512, 256, false, true>(mq, mk, mv, pp, pl, st);
-  return bf16 ? launch_prefill<512, 256, true>(mq, mk, mv, pp, pl, st)
-              : launch_prefill<512, 256, false>(mq, mk, mv, pp, pl, st);
+  return bf16 ? launch_prefill_ab<true>(mq, mk, mv, pp, pl, st)
+              : launch_prefill_ab<false>(mq, mk, mv, pp, pl, st);
 }
 
 }  // namespace

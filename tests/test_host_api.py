@@ -140,9 +140,13 @@ def test_plan_extend_takes_decode_path(lib):
 
 
 def test_plan_prefill(lib):
+    # d = 512: SM pairs split the two matmuls (one CTA S and softmax, the
+    # other O and PV); a work item is 128 query rows of one head, all of d_v
     pl = binding.plan(2, 16, 1, 4096, 4096, 512, 512, num_sms=148)
-    assert pl["path"] == 0 and pl["dv_parts"] == 2 and pl["workspace_bytes"] == 0
-    assert pl["grid_ctas"] == 148  # persistent: one CTA per SM walks the 2048 work items
+    assert pl["path"] == 0 and pl["dv_parts"] == 1 and pl["workspace_bytes"] == 0
+    assert pl["grid_ctas"] == 148  # persistent: 74 pairs walk the 1024 work items
+    pl = binding.plan(1, 3, 1, 129, 150, 512, 512, num_sms=148)
+    assert pl["grid_ctas"] == 2 * 6  # 6 items (2 q tiles x 3 heads), one pair each
     pl = binding.plan(1, 64, 8, 8192, 8192, 128, 128, num_sms=148)
     assert pl["dv_parts"] == 1 and pl["grid_ctas"] == 148
     pl = binding.plan(1, 2, 1, 100, 100, 128, 128, num_sms=148)
