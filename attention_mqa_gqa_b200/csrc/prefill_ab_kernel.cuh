@@ -10,8 +10,9 @@
 //   CTA 0 ("scores"):  Q (bf16/fp16) in TMEM columns 256..511, copied there
 //       once per item; S[128 x 128 keys] = Q K^T by TMEM-operand UMMAs into
 //       two S buffers (columns 0..255); the online softmax (four threads per
-//       query row) turns each 64-key half of S into P and sends it, with the
-//       rows' rescale factors, into CTA 1's shared memory by st.async.
+//       query row) turns each 64-key half of S into P, writes it into a
+//       local staging buffer and ships it to CTA 1's shared memory with
+//       bulk copies (four 4 KB copies per half, one per 32-row quarter).
 //   CTA 1 ("output"):  O[128 x 512] in all of its TMEM; O += P V over each
 //       64-key half (two UMMAs of N = 256); when a row's running maximum
 //       was raised it rescales O in TMEM first; at the end of the item
@@ -30,10 +31,14 @@
 //   CTA 1: warp 0 lane 0 copies V; warp 1 issues the PV UMMAs and posts
 //       events (rescale, end of item) to warps 2-17, which rescale O or
 //       write the output.
-// Cross-CTA traffic: P, rescale factors and row sums by st.async (bytes
-// counted on a CTA 1 mbarrier); "P buffer free" by tcgen05.commit multicast
-// from CTA 1's MMA issuer.  All waits are bounded; the two CTAs meet in a
-// hardware cluster barrier only after both have left every loop.
+// Cross-CTA traffic: P by cp.async.bulk from CTA 0's staging buffers (on
+// this part a bulk copy moves shared memory to the peer SM about twice as
+// fast as st.async), rescale factors, partial row sums and row maxima by
+// st.async (all bytes counted on CTA 1 mbarriers); "P buffer free" by
+// tcgen05.commit multicast from CTA 1's MMA issuer; "staging buffer read"
+// and "row sums read" by relaxed remote arrivals from CTA 1.  All waits are
+// bounded; the two CTAs meet in a hardware cluster barrier only after both
+// have left every loop.
 #pragma once
 
 #include "prefill_kernel.cuh"
@@ -48,32 +53,49 @@ struct PrefillABTraits {
   static constexpr int SLOT = 65536;             // one copy: 4 chunks x 128 rows or 8 x 64
   static constexpr int CHUNK_Q = 16384;          // [128 rows x 64 columns] of Q or K
   static constexpr int CHUNK_V = 8192;           // [64 keys x 64 columns] of V
-  static constexpr int RING = 3;
+  static constexpr int RING = 3;                 // CTA 0: Q/K copies in flight
+  static constexpr int RING_V = 2;               // CTA 1: V copies in flight
+  static constexpr int NPB = 4;                  // CTA 1: P half buffers (two tiles)
   static constexpr int SPLIT = 4;                // scores CTA: threads per q row
   static constexpr int KS = HT / SPLIT;          // keys per thread per half tile (16)
   static constexpr int SOFTMAX_THREADS = 128 * SPLIT;
   static constexpr int WORK_WARPS = SOFTMAX_THREADS / 32;  // warps 2.. of either CTA
-  static constexpr int THREADS = 64 + SOFTMAX_THREADS;
+  static constexpr int RELAY_WARP = 2 + WORK_WARPS;         // CTA 1: P arrivals -> CTA 0
+  static constexpr int THREADS = 64 + SOFTMAX_THREADS + 32;
   static constexpr int PH_BYTES = TILE * HT * 2;           // one P half: 16 KB
-  static constexpr int PMSG_BYTES = PH_BYTES + TILE * 4;   // P half + rescale factors
+  // bytes landing in P buffer b: a tile's first half (even b) comes with the
+  // rows' rescale factors, its second half (odd b) needs none
+  static constexpr int PMSG_BYTES = PH_BYTES + TILE * 4;
+  __host__ __device__ static constexpr int pmsg_bytes(int b) { return (b & 1) ? PH_BYTES : PMSG_BYTES; }
+  static constexpr int PQ_BYTES = PH_BYTES / 4;            // one 32-row quarter of a P half
+  static constexpr int L_BYTES = (SPLIT + 1) * TILE * 4;   // partial row sums + row maxima
+  // CTA 0: ring of RING slots, row-maximum exchange, two P staging buffers.
+  // CTA 1: ring of RING_V slots, the P half buffers (K-major, 128-byte
+  // swizzle) where CTA 0's third slot lies, rescale factors, row sums.  The
+  // base must be 1024-byte aligned (checked at entry): there is no slack.
   static constexpr int OFF_RING = 0;
-  // CTA 1: P halves [2] (K-major, 128-byte swizzle); CTA 0: row exchange
-  static constexpr int OFF_P = OFF_RING + RING * SLOT;
-  static constexpr int OFF_ALPHA = OFF_P + 2 * PH_BYTES;   // CTA 1: float [2][128]
-  static constexpr int OFF_L = OFF_ALPHA + 2 * TILE * 4;   // CTA 1: float [128] row sums
-  static constexpr int OFF_EV = OFF_L + TILE * 4;          // CTA 1: event {type, arg0, arg1, arg2}
+  static constexpr int OFF_P = OFF_RING + RING_V * SLOT;
+  static constexpr int OFF_SIDE = OFF_RING + RING * SLOT;
+  static constexpr int OFF_XCH = OFF_SIDE;                 // CTA 0: float [SPLIT][128]
+  static constexpr int OFF_STAGE = OFF_SIDE + SPLIT * TILE * 4;  // CTA 0: [2 halves][PH_BYTES]
+  static constexpr int OFF_ALPHA = OFF_SIDE;               // CTA 1: float [NPB][128]
+  static constexpr int OFF_L = OFF_ALPHA + NPB * TILE * 4; // CTA 1: float [SPLIT][128] partial sums
+  static constexpr int OFF_M = OFF_L + SPLIT * TILE * 4;   // CTA 1: float [128] row maxima (log2)
+  static constexpr int OFF_EV = OFF_STAGE + 2 * PH_BYTES;  // CTA 1: event {type, arg0, arg1, arg2}
   static constexpr int OFF_FLAGS = OFF_EV + 16;            // int [4]: abort, tmem
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
-  // full[3] empty[3] s_full[2] s_free[2] q_cp p_free[2] p_full[2] o_item
-  // o_sync ev_go ev_done l_full drain (the same layout in both CTAs: p_free
-  // is reached by a multicast commit, the others by mapa)
-  static constexpr int NBAR = 2 * RING + 2 + 2 + 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1 + 1;
-  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
-  static constexpr int XR = 2;                   // row exchange rounds (CTA 0)
+  // full[3] empty[3] s_full[2] s_free[2] q_cp p_free[4] p_full[4] o_item
+  // o_sync ev_go ev_done l_full drain stage_free l_free (the same layout
+  // in both CTAs: p_free is reached by a multicast commit, the others by
+  // mapa)
+  static constexpr int NBAR = 2 * RING + 2 + 2 + 1 + 2 * NPB + 1 + 1 + 1 + 1 + 1 + 1 + 1 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8;
   static constexpr int TMEM_S = 0;               // CTA 0: S buffers, 128 columns each
   static constexpr int TMEM_Q = 256;             // CTA 0: Q, 8 columns per 16-element K step
   static constexpr int TMEM_O = 0;               // CTA 1: O, 512 columns
-  static_assert(XR * SPLIT * TILE * 4 <= 2 * PH_BYTES, "row exchange fits the P region");
+  static_assert(OFF_P + NPB * PH_BYTES == OFF_SIDE, "CTA 1's P buffers end where CTA 0's ring does");
+  static_assert(OFF_M + TILE * 4 <= OFF_EV && OFF_STAGE % 1024 == 0, "side buffers");
+  static_assert(NPB % 2 == 0, "a tile's two halves take consecutive P buffers");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -93,12 +115,25 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  // The layout fills the shared memory limit with no alignment slack: a base
+  // that is not 1024-byte aligned (never seen: the dynamic window starts
+  // aligned) is reported instead of used.  Both CTAs see the same base and
+  // leave before any cluster barrier.
+  if (smem != smem_raw) {
+    if (threadIdx.x == 0) {
+      atomicCAS(&g_attn_error, 0u, 1u | (89u << 8));
+      atomicOr(&g_attn_error, 1u);
+    }
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t ring = sbase + T::OFF_RING;
   const uint32_t pbuf = sbase + T::OFF_P;
-  float* xch = reinterpret_cast<float*>(smem + T::OFF_P);          // CTA 0
+  float* xch = reinterpret_cast<float*>(smem + T::OFF_XCH);        // CTA 0
+  const uint32_t stage = sbase + T::OFF_STAGE;                      // CTA 0
   float* alpha_sm = reinterpret_cast<float*>(smem + T::OFF_ALPHA);  // CTA 1
   float* l_sm = reinterpret_cast<float*>(smem + T::OFF_L);          // CTA 1
+  float* m_sm = reinterpret_cast<float*>(smem + T::OFF_M);          // CTA 1
   volatile int* ev = reinterpret_cast<volatile int*>(smem + T::OFF_EV);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_FLAGS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_FLAGS + 4);
@@ -108,14 +143,16 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
   const uint32_t s_full = bar0 + 8u * (2 * T::RING);  // [2] CTA 0
   const uint32_t s_free = s_full + 16;                // [2] CTA 0
   const uint32_t q_cp = s_free + 16;                  // CTA 0: Q in TMEM
-  const uint32_t p_free = q_cp + 8;                   // [2] CTA 0: P half buffer free in CTA 1
-  const uint32_t p_full = p_free + 16;                // [2] CTA 1: P half + factors landed
-  const uint32_t o_item = p_full + 16;                // CTA 1: an item's last PV completed
+  const uint32_t p_free = q_cp + 8;                   // [NPB] CTA 0: P half buffer free in CTA 1
+  const uint32_t p_full = p_free + 8 * T::NPB;        // [NPB] CTA 1: P half + factors landed
+  const uint32_t o_item = p_full + 8 * T::NPB;        // CTA 1: an item's last PV completed
   const uint32_t o_sync = o_item + 8;                 // CTA 1: every PV issued so far completed
   const uint32_t ev_go = o_sync + 8;                  // CTA 1: event posted
   const uint32_t ev_done = ev_go + 8;                 // CTA 1: event handled
-  const uint32_t l_full = ev_done + 8;                // CTA 1: row sums landed
+  const uint32_t l_full = ev_done + 8;                // CTA 1: row sums and maxima landed
   const uint32_t drain = l_full + 8;
+  const uint32_t stage_free = drain + 8;              // CTA 0: the staged tile has landed in CTA 1
+  const uint32_t l_free = stage_free + 8;             // CTA 0: CTA 1 has read the row sums
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -128,6 +165,8 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
       mbar_init(s_free + 8 * i, T::WORK_WARPS);
+    }
+    for (int i = 0; i < T::NPB; ++i) {
       mbar_init(p_free + 8 * i, 1);
       mbar_init(p_full + 8 * i, 1);
     }
@@ -138,12 +177,13 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     mbar_init(ev_done, T::WORK_WARPS);
     mbar_init(l_full, 1);
     mbar_init(drain, 1);
+    mbar_init(stage_free, 1);
+    mbar_init(l_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if (cr == 1) {  // the first two P halves and the first item's row sums
-      mbar_arrive_expect_tx(p_full, T::PMSG_BYTES);
-      mbar_arrive_expect_tx(p_full + 8, T::PMSG_BYTES);
-      mbar_arrive_expect_tx(l_full, T::TILE * 4);
+    if (cr == 1) {  // the first NPB P halves and the first item's row sums
+      for (int i = 0; i < T::NPB; ++i) mbar_arrive_expect_tx(p_full + 8 * i, T::pmsg_bytes(i));
+      mbar_arrive_expect_tx(l_full, T::L_BYTES);
     }
   }
   if (warp == 1) {
@@ -203,7 +243,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
           mbar_arrive_expect_tx(full_bar(grp), T::SLOT);
           tma_load_5d(ring + grp * T::SLOT, &tmV, full_bar(grp), 0, win0 + hh * T::HT, 0, it.kvh,
                       it.b, pol_v);
-          if (++grp == T::RING) { grp = 0; ph ^= 1u; }
+          if (++grp == T::RING_V) { grp = 0; ph ^= 1u; }
         }
       }
     }
@@ -284,10 +324,22 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     uint32_t ph = 0;
     bool ok = true;
     int h = 0, ne = 0, nsync = 0;  // half tiles, events posted, o_sync phases
+    const uint32_t l_free_0 = mapa_shared(l_free, 0);
+    bool out_pending = false;  // an item's output event not yet seen handled
+    // wait until the last event posted was handled; once an item's output
+    // has been written, its row sums are read: CTA 0 may send the next ones
+    auto wait_done = [&](uint32_t id) {
+      ok = mbar_wait_warp(ev_done, (ne - 1) & 1, abort_flag, tmo, id);
+      if (ok && out_pending) {
+        if (lane == 0) mbar_arrive_remote_relaxed(l_free_0);
+        __syncwarp();
+        out_pending = false;
+      }
+    };
     // one event at a time: wait until the previous one was handled
     auto post = [&](int type, int a0, int a1, int a2) {
       if (!ok) return;
-      if (ne > 0) ok = mbar_wait_warp(ev_done, (ne - 1) & 1, abort_flag, tmo, 77);
+      if (ne > 0) wait_done(77);
       if (!ok) return;
       if (lane == 0) {
         ev[0] = type;
@@ -307,14 +359,15 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
       }
       for (int t = 0; t < it.ntiles && ok; ++t) {
         for (int hh = 0; hh < 2 && ok; ++hh, ++h) {
-          const int pb = h & 1;
+          const int pb = h % T::NPB;
           const bool first = t == 0 && hh == 0;
-          ok = mbar_wait_warp_cluster(p_full + 8 * pb, (h >> 1) & 1, abort_flag, tmo, 78);
+          ok = mbar_wait_warp_cluster(p_full + 8 * pb, (h / T::NPB) & 1, abort_flag, tmo, 78);
           if (!ok) break;
-          // rows whose running maximum was raised: O *= alpha first (the
+          // rows whose running maximum was raised at this tile: O *= alpha
+          // before its first half (the factors come with that half; the
           // first half of an item overwrites O, so needs none)
           bool rescale = false;
-          if (!first) {
+          if (!first && hh == 0) {
             const float4 a4 = *reinterpret_cast<const float4*>(alpha_sm + pb * T::TILE + 4 * lane);
             rescale = __any_sync(0xffffffffu, a4.x != 1.f || a4.y != 1.f || a4.z != 1.f || a4.w != 1.f);
           }
@@ -325,12 +378,12 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
             ok = mbar_wait_warp(o_sync, nsync & 1, abort_flag, tmo, 79);
             ++nsync;
             post(AB_EV_RESCALE, pb, 0, 0);
-            if (ok) ok = mbar_wait_warp(ev_done, (ne - 1) & 1, abort_flag, tmo, 80);
+            if (ok) wait_done(80);
             if (!ok) break;
             tc_fence_after();
           }
           if (first && ne > 0) {  // the previous event (an item's output) read O out of TMEM
-            ok = mbar_wait_warp(ev_done, (ne - 1) & 1, abort_flag, tmo, 81);
+            wait_done(81);
             if (!ok) break;
             tc_fence_after();
           }
@@ -339,8 +392,8 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
           tc_fence_after();
           fence_proxy_async_smem();  // the st.async P rows, for the MMA's operand reads
           if (elect_one()) {
-            // the next use of this P buffer (half h + 2)
-            mbar_arrive_expect_tx(p_full + 8 * pb, T::PMSG_BYTES);
+            // the next use of this P buffer (half h + NPB)
+            mbar_arrive_expect_tx(p_full + 8 * pb, T::pmsg_bytes(pb));
             // A = P half: K-major, 128-byte swizzle, 32 bytes per K step.
             // B = V half [8 chunks][64 keys][64 columns]: MN-major, 128-byte
             // swizzle, 64-column chunks 8 KB apart (LBO), 8-key groups 1024
@@ -360,14 +413,17 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
             if (t == it.ntiles - 1 && hh == 1) umma_commit(o_item);  // the item's O is complete
           }
           __syncwarp();
-          if (++grp == T::RING) { grp = 0; ph ^= 1u; }
+          if (++grp == T::RING_V) { grp = 0; ph ^= 1u; }
         }
       }
-      if (ok) post(AB_EV_OUTPUT, L, h - 1, 0);
+      if (ok) {
+        post(AB_EV_OUTPUT, L, h - 1, 0);
+        out_pending = true;
+      }
     }
     post(AB_EV_STOP, 0, 0, 0);
     if (!ok) *abort_flag = 1;
-  } else if (cr == 0 && warp >= 2) {
+  } else if (cr == 0 && warp >= 2 && warp < T::RELAY_WARP) {
     // ---------------------------------------------------- CTA 0: softmax
     // SPLIT threads per q row: warps with the same warp % 4 share a TMEM lane
     // quarter; quarter-mate qd owns keys [KS qd, KS qd + KS) of each 64-key
@@ -385,100 +441,160 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     const uint32_t pbuf_1 = mapa_shared(pbuf, 1);
     const uint32_t alpha_1 = mapa_shared(smem_u32(alpha_sm), 1);
     const uint32_t l_1 = mapa_shared(smem_u32(l_sm), 1);
+    const uint32_t m_1 = mapa_shared(smem_u32(m_sm), 1);
     const uint32_t l_full_1 = mapa_shared(l_full, 1);
-    bool ok = true;
-    int j = 0, h = 0, xr = 0;
+    // this thread's two 16-byte units of a P half row, at the same offsets
+    // in a staging buffer and in CTA 1's P buffer (K-major, 128-byte
+    // swizzle: unit v of row r at 128 r + ((v ^ (r & 7)) * 16)); the 32 rows
+    // of a lane quarter are one contiguous 4 KB block
+    const uint32_t pofs0 = row * 128 + (((2 * qd) ^ (row & 7)) << 4);
+    const uint32_t pofs1 = row * 128 + (((2 * qd + 1) ^ (row & 7)) << 4);
+    static_assert(KS == 16, "two 16-byte units of P per thread and half");
+    bool ok = true;   // this warp's waits
+    bool gok = true;  // the group's, from its last barrier
+    int j = 0, h = 0, nitem = 0;
     for (int L = item0; L < p.n_items; L += istride) {
       const PrefillItem it = prefill_item(p, L, 0);
+      if (it.ntiles == 0) continue;  // CTA 1 writes the empty item
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
       lim = max(0, min(it.skv, lim));
       float m_used = -INFINITY;  // log2-domain running max, the same in the group
-      float l = 0.f;
+      float l = 0.f;             // this thread's share of the row sum
       for (int t = 0; t < it.ntiles; ++t, ++j) {
         const int sb = j & 1;
         if (ok) ok = mbar_wait_warp(s_full + 8 * sb, (j >> 1) & 1, &own_abort, tmo, 83);
         if (ok) tc_fence_after();
         const int tile0 = t * T::KT;
         const int win0 = min(tile0, it.skv - T::KT);
-        for (int hh = 0; hh < 2; ++hh, ++h) {
-          const int pb = h & 1;
-          float s[KS];
-          float mx = -INFINITY;
-          const int key0 = win0 + hh * T::HT + qd * KS;
-          if (ok) {
-            tmem_ld<KS>(tmem + lane_base + T::TMEM_S + sb * 128 + hh * T::HT + qd * KS, s);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < KS; ++e) {
-              const int key = key0 + e;
-              const bool vis = key >= tile0 && key < lim;
-              s[e] = vis ? s[e] * p.scale_log2 : -INFINITY;
-              mx = fmaxf(mx, s[e]);
-            }
-          }
-          float* xb = xch + (xr & 1) * (T::SPLIT * T::TILE);
-          ++xr;
-          xb[qd * T::TILE + row] = mx;
-          ok = group_and(ok);
-          float tm = -INFINITY;
-#pragma unroll
-          for (int k = 0; k < T::SPLIT; ++k) tm = fmaxf(tm, xb[k * T::TILE + row]);
-          // lazy raise (threshold 8 in log2 units): the weights stay <= 256
-          const bool need = tm > m_used + 8.f;
-          const float mn = need ? tm : m_used;
-          const float alpha = need ? ex2(m_used - mn) : 1.f;  // m_used = -inf: 0
-          m_used = mn;
-          l *= alpha;
-          // CTA 1's P buffer pb was last read by PV(h - 2)
-          if (ok && h >= 2)
-            ok = mbar_wait_warp_cluster(p_free + 8 * pb, ((h >> 1) - 1) & 1, &own_abort, tmo, 84);
-          if (ok) {
-            uint32_t u[KS / 2];
-            // an invisible key's weight is exactly 0 (ex2(-inf) = +0); a row
-            // with no visible key yet keeps m_used = -inf and all weights 0
-            const float mu = m_used == -INFINITY ? 0.f : m_used;
-#pragma unroll
-            for (int e = 0; e < KS; e += 2) {
-              const float p0 = ex2(s[e] - mu);
-              const float p1 = ex2(s[e + 1] - mu);
-              l += p0 + p1;
-              u[e / 2] = pack2(p0, p1, BF16);
-            }
-            // P half, K-major 128-byte swizzle: row r at 128 r, 16-byte unit
-            // (8 keys) v at ((v ^ (r & 7)) * 16)
-            const uint32_t prow = pbuf_1 + pb * T::PH_BYTES + row * 128;
-            const uint32_t bar = p_full_1 + 8 * pb;
-#pragma unroll
-            for (int v = 0; v < KS / 8; ++v) {
-              const int unit = qd * (KS / 8) + v;
-              st_async_v4(prow + ((unit ^ (row & 7)) << 4), u[4 * v], u[4 * v + 1], u[4 * v + 2],
-                          u[4 * v + 3], bar);
-            }
-            if (qd == 0) st_async_f32(alpha_1 + (pb * T::TILE + row) * 4, alpha, bar);
-          }
+        // both halves of this thread's slice of the tile: keys win0 + 64 hh +
+        // KS qd + e (a shifted last window's keys below tile0 belong to the
+        // previous tile)
+        float s[2 * KS];
+        float mx = -INFINITY;
+        // a tile wholly inside [0, lim) for this row: no mask, and a quarter
+        // of its exponentials go to the FMA pipe
+        const bool whole = win0 == tile0 && tile0 + T::KT <= lim;
+        if (ok) {
+          tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + qd * KS, *reinterpret_cast<float(*)[16]>(s));
+          tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + T::HT + qd * KS,
+                    *reinterpret_cast<float(*)[16]>(s + KS));
+          tmem_wait_ld();
         }
-        // S buffer sb has been read
+        // S buffer sb has been read: the next S may go there
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free + 8 * sb);
-      }
-      // row sum over the group, to CTA 1 with the row's LSE written here
-      float* xb = xch + (xr & 1) * (T::SPLIT * T::TILE);
-      ++xr;
-      xb[qd * T::TILE + row] = l;
-      ok = group_and(ok);
-      if (!ok) break;
-      float ltot = 0.f;
+        if (ok) {
+          // raw scores here (scale > 0 keeps the order)
+          if (whole) {
 #pragma unroll
-      for (int k = 0; k < T::SPLIT; ++k) ltot += xb[k * T::TILE + row];
-      if (it.ntiles > 0 && qd == 0) st_async_f32(l_1 + row * 4, ltot, l_full_1);
-      if (qd == 0 && p.lse && qi < p.Sq)
-        p.lse[((int64_t)it.b * p.Hq + it.h) * p.Sq + qi] =
-            ltot > 0.f ? (m_used + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
+            for (int e = 0; e < 2 * KS; e += 2) mx = fmaxf(mx, fmaxf(s[e], s[e + 1]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 2 * KS; ++e) {
+              const int key = win0 + (e / KS) * T::HT + qd * KS + (e % KS);
+              s[e] = (key >= tile0 && key < lim) ? s[e] : -INFINITY;
+              mx = fmaxf(mx, s[e]);
+            }
+          }
+        }
+        // the row maximum over the tile's 128 keys.  One exchange buffer is
+        // enough: every thread has read it before it passes the barriers of
+        // this tile's halves, and it is written again only after them.
+        xch[qd * T::TILE + row] = mx;
+        gok = group_and(ok);
+        ok = gok;
+        if (!gok) break;
+        float tm = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < T::SPLIT; ++k) tm = fmaxf(tm, xch[k * T::TILE + row]);
+        tm *= p.scale_log2;
+        // lazy raise (threshold 8 in log2 units): the weights stay <= 256
+        const bool need = tm > m_used + 8.f;
+        const float mn = need ? tm : m_used;
+        const float alpha = need ? ex2(m_used - mn) : 1.f;  // m_used = -inf: 0
+        m_used = mn;
+        l *= alpha;
+        // an invisible key's weight is exactly 0 (ex2(-inf) = +0); a row
+        // with no visible key yet keeps m_used = -inf and all weights 0
+        const float neg_mu = m_used == -INFINITY ? 0.f : -m_used;
+        // both halves' P, then one staging write, one barrier and the
+        // copies of the whole tile
+        uint32_t u[2][KS / 2];
+        if (whole) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < KS; e += 2) {
+              const float p0 = ex2(fmaf(s[hh * KS + e], p.scale_log2, neg_mu));
+              const float x1 = fmaf(s[hh * KS + e + 1], p.scale_log2, neg_mu);
+              const float p1 = (e & 2) ? ex2_fma(x1) : ex2(x1);
+              l += p0 + p1;
+              u[hh][e / 2] = pack2(p0, p1, BF16);
+            }
+        } else {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int e = 0; e < KS; e += 2) {
+              const float p0 = ex2(fmaf(s[hh * KS + e], p.scale_log2, neg_mu));
+              const float p1 = ex2(fmaf(s[hh * KS + e + 1], p.scale_log2, neg_mu));
+              l += p0 + p1;
+              u[hh][e / 2] = pack2(p0, p1, BF16);
+            }
+        }
+        // the staging buffer last held tile j - 1: CTA 1 reports once it has
+        // seen both of its halves land
+        if (ok && j >= 1) ok = mbar_wait_warp(stage_free, (j - 1) & 1, &own_abort, tmo, 91);
+        if (ok) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            st_shared_v4(stage + hh * T::PH_BYTES + pofs0, u[hh][0], u[hh][1], u[hh][2], u[hh][3]);
+            st_shared_v4(stage + hh * T::PH_BYTES + pofs1, u[hh][4], u[hh][5], u[hh][6], u[hh][7]);
+          }
+          fence_proxy_async_smem();  // for the bulk copies' reads
+        }
+        gok = group_and(ok);
+        ok = gok;
+        if (!gok) break;
+        // The quarter's two copies and the rescale factors of the tile's
+        // first half, one job per warp of the group: qd = 0 copies half 0,
+        // qd = 1 half 1, qd = 2 sends the factors.  CTA 1's P buffer pb +
+        // hh was last read by PV(h + hh - NPB).  A failed wait here reaches
+        // the group at its next barrier.
+        const int pb = h % T::NPB;  // h is even, NPB too: pb + 1 is the next buffer
+        if (qd < 3) {
+          const int hh = qd & 1;
+          if (ok && h >= T::NPB)
+            ok = mbar_wait_warp_cluster(p_free + 8 * (pb + hh), ((h / T::NPB) - 1) & 1, &own_abort, tmo, 84);
+          if (ok) {
+            const uint32_t bar = p_full_1 + 8 * (pb + hh);
+            if (qd < 2) {
+              if (lane == 0)
+                bulk_copy_to_peer(pbuf_1 + (pb + hh) * T::PH_BYTES + wq * T::PQ_BYTES,
+                                  stage + hh * T::PH_BYTES + wq * T::PQ_BYTES, T::PQ_BYTES, bar);
+            } else {
+              // O's rescale factor before the tile's first PV
+              st_async_f32(alpha_1 + (pb * T::TILE + row) * 4, alpha, bar);
+            }
+          }
+        }
+        h += 2;
+      }
+      if (!gok) break;  // the same in the whole group (set by its last barrier)
+      // the partial row sums and the row maximum, once CTA 1 has read the
+      // previous item's.  A failed wait only clears `ok`: the group learns
+      // of it at its next barrier.
+      if (ok && nitem > 0) ok = mbar_wait_warp_cluster(l_free, (nitem - 1) & 1, &own_abort, tmo, 92);
+      ++nitem;
+      if (ok) {
+        st_async_f32(l_1 + (qd * T::TILE + row) * 4, l, l_full_1);
+        if (qd == 0) st_async_f32(m_1 + row * 4, m_used, l_full_1);
+      }
     }
     if (!ok) *abort_flag = 1;
-  } else if (cr == 1 && warp >= 2) {
+  } else if (cr == 1 && warp >= 2 && warp < T::RELAY_WARP) {
     // ---------------------------------------------------- CTA 1: rescale, output
     // Four threads per row (warps with the same warp % 4 share a TMEM lane
     // quarter), each owning 128 of the row's 512 output columns.
@@ -522,52 +638,80 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
       } else {  // AB_EV_OUTPUT, AB_EV_EMPTY: O / l -> out for item a0
         const PrefillItem it = prefill_item(p, a0, 0);
         const int qi = it.q0 + row;
-        float inv = 0.f;
+        float inv = 0.f, lse = -INFINITY;
         if (type == AB_EV_OUTPUT) {
           ok = mbar_wait_warp(o_item, nl & 1, &own_abort, tmo, 86) &&
                mbar_wait_warp_cluster(l_full, nl & 1, &own_abort, tmo, 87);
           if (ok) {
             tc_fence_after();
-            const float lt = l_sm[row];
+            float lt = 0.f;  // the row sum from the scores CTA's SPLIT shares
+#pragma unroll
+            for (int k = 0; k < T::SPLIT; ++k) lt += l_sm[k * T::TILE + row];
             inv = lt > 0.f ? 1.f / lt : 0.f;
+            if (lt > 0.f) lse = (m_sm[row] + __log2f(lt)) * 0.69314718055994531f;
           }
         }
+        if (ok && qd == 0 && p.lse && qi < p.Sq)
+          p.lse[((int64_t)it.b * p.Hq + it.h) * p.Sq + qi] = lse;
         if (ok) {  // warp-uniform: the TMEM loads are warp-collective
           uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
                           ((int64_t)it.b * p.o_sb + (int64_t)it.h * p.o_sh + (int64_t)qi * p.o_ss +
                            qd * HC) * 2;
 #pragma unroll 1
-          for (int c0 = 0; c0 < HC; c0 += 16) {
-            float o[16];
+          for (int c0 = 0; c0 < HC; c0 += 32) {
+            float o[32];
             if (type == AB_EV_OUTPUT) {
-              tmem_ld16(tmem + lane_base + T::TMEM_O + qd * HC + c0, o);
+              tmem_ld16(tmem + lane_base + T::TMEM_O + qd * HC + c0, *reinterpret_cast<float(*)[16]>(o));
+              tmem_ld16(tmem + lane_base + T::TMEM_O + qd * HC + c0 + 16,
+                        *reinterpret_cast<float(*)[16]>(o + 16));
               tmem_wait_ld();
             } else {
 #pragma unroll
-              for (int c = 0; c < 16; ++c) o[c] = 0.f;
+              for (int c = 0; c < 32; ++c) o[c] = 0.f;
             }
             if (qi < p.Sq) {  // rows past Sq (a partial last q tile) are not stored
-              uint32_t u[8];
+              uint32_t u[16];
 #pragma unroll
-              for (int c = 0; c < 8; ++c) u[c] = pack2(o[2 * c] * inv, o[2 * c + 1] * inv, BF16);
+              for (int c = 0; c < 16; ++c) u[c] = pack2(o[2 * c] * inv, o[2 * c + 1] * inv, BF16);
               uint4* dst = reinterpret_cast<uint4*>(orow + c0 * 2);
-              dst[0] = make_uint4(u[0], u[1], u[2], u[3]);
-              dst[1] = make_uint4(u[4], u[5], u[6], u[7]);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
             }
           }
         }
         if (type == AB_EV_OUTPUT) {
           tc_fence_before();
-          // row sums consumed: arm the next item's (every thread has read them
-          // once all warps arrive on ev_done, which the next item's first PV
-          // waits for, before CTA 0 can send them)
-          if (ok && threadIdx.x == 64) mbar_arrive_expect_tx(l_full, T::TILE * 4);
+          // row sums consumed: arm the next item's (CTA 0 sends them only
+          // after the MMA issuer has seen every warp arrive on ev_done and
+          // told it so through l_free)
+          if (ok && threadIdx.x == 64) mbar_arrive_expect_tx(l_full, T::L_BYTES);
           ++nl;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(ev_done);
       if (!ok) break;
+    }
+    if (!ok) *abort_flag = 1;
+  } else if (cr == 1 && warp == T::RELAY_WARP) {
+    // ---------------------------------------------------- CTA 1: P arrivals -> CTA 0
+    // Watches the P buffers fill, in order, and tells CTA 0 as soon as both
+    // halves of a tile have landed, so that its staging buffer can take the
+    // next tile.  (The MMA issuer waits on the same barriers; a phase cannot
+    // complete twice before this warp sees it, since the copies that would
+    // complete it next come from a staging buffer this warp must free first.)
+    const uint32_t stage_free_0 = mapa_shared(stage_free, 0);
+    bool ok = true;
+    int h = 0;
+    for (int L = item0; L < p.n_items && ok; L += istride) {
+      const PrefillItem it = prefill_item(p, L, 0);
+      for (int t = 0; t < it.ntiles && ok; ++t, h += 2) {
+        ok = mbar_wait_warp_cluster(p_full + 8 * (h % T::NPB), (h / T::NPB) & 1, abort_flag, tmo, 93) &&
+             mbar_wait_warp_cluster(p_full + 8 * ((h + 1) % T::NPB), ((h + 1) / T::NPB) & 1, abort_flag,
+                                    tmo, 93);
+        if (ok && lane == 0) mbar_arrive_remote_relaxed(stage_free_0);
+        __syncwarp();
+      }
     }
     if (!ok) *abort_flag = 1;
   }

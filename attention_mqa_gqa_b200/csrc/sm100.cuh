@@ -64,6 +64,23 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 64: Cody-Waite range reduction (x = n + f,
+// n = round(x) by the 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]) and a
+// cubic for 2^f fitted by a Remez exchange on the relative error (max
+// 7.5e-5), scaled by adding n to the exponent field.  x is clamped at -125,
+// so the result is never below 2^-125.5 (not 0): callers use it where
+// every key is visible.  Offloads part of a softmax's exponentials from the
+// SFU, whose rate is an eighth of the FMA pipe's.
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float q = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  q = fmaf(q, f, 0.6932609677314758f);
+  q = fmaf(q, f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -547,6 +564,18 @@ __device__ __forceinline__ void st_async_f32(uint32_t raddr, float v, uint32_t r
                    raddr),
                "r"(__float_as_uint(v)), "r"(rbar)
                : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory to a peer CTA's (`dst` and `rbar` from
+// mapa); the bytes are counted on the peer's mbarrier `rbar`.  The source
+// may be reused only once that barrier's phase has completed.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes,
+                                                  uint32_t rbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(rbar)
+      : "memory");
 }
 
 // try_wait with acquire at cluster scope (for phases completed by arrivals
