@@ -56,40 +56,37 @@ struct PrefillABTraits {
   static constexpr int RING = 3;                 // CTA 0: Q/K copies in flight
   static constexpr int RING_V = 2;               // CTA 1: V copies in flight
   static constexpr int NPB = 4;                  // CTA 1: P half buffers (two tiles)
-  static constexpr int SPLIT = 4;                // scores CTA: threads per q row
-  static constexpr int KS = HT / SPLIT;          // keys per thread per half tile (16)
-  static constexpr int SOFTMAX_THREADS = 128 * SPLIT;
-  static constexpr int WORK_WARPS = SOFTMAX_THREADS / 32;  // warps 2.. of either CTA
+  static constexpr int SM_WARPS = 8;             // CTA 0: softmax warps 2..9, a q row per thread and half
+  static constexpr int SPLIT = 4;                // CTA 1: output threads per q row
+  static constexpr int WORK_WARPS = 4 * SPLIT;   // CTA 1: output warps 2..17
   static constexpr int RELAY_WARP = 2 + WORK_WARPS;         // CTA 1: P arrivals -> CTA 0
-  static constexpr int THREADS = 64 + SOFTMAX_THREADS + 32;
+  static constexpr int THREADS = 64 + 32 * WORK_WARPS + 32;
   static constexpr int PH_BYTES = TILE * HT * 2;           // one P half: 16 KB
   // bytes landing in P buffer b: a tile's first half (even b) comes with the
   // rows' rescale factors, its second half (odd b) needs none
   static constexpr int PMSG_BYTES = PH_BYTES + TILE * 4;
   __host__ __device__ static constexpr int pmsg_bytes(int b) { return (b & 1) ? PH_BYTES : PMSG_BYTES; }
   static constexpr int PQ_BYTES = PH_BYTES / 4;            // one 32-row quarter of a P half
-  static constexpr int L_BYTES = (SPLIT + 1) * TILE * 4;   // partial row sums + row maxima
-  // CTA 0: ring of RING slots, row-maximum exchange, two P staging buffers.
-  // CTA 1: ring of RING_V slots, the P half buffers (K-major, 128-byte
-  // swizzle) where CTA 0's third slot lies, rescale factors, row sums.  The
-  // base must be 1024-byte aligned (checked at entry): there is no slack.
+  static constexpr int L_BYTES = 3 * TILE * 4;             // the halves' row sums + row maxima
+  // CTA 0: ring of RING slots, two P half staging buffers.  CTA 1: ring of
+  // RING_V slots, the P half buffers (K-major, 128-byte swizzle) where CTA
+  // 0's third slot lies, rescale factors, row sums and maxima.
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_P = OFF_RING + RING_V * SLOT;
   static constexpr int OFF_SIDE = OFF_RING + RING * SLOT;
-  static constexpr int OFF_XCH = OFF_SIDE;                 // CTA 0: float [SPLIT][128]
-  static constexpr int OFF_STAGE = OFF_SIDE + SPLIT * TILE * 4;  // CTA 0: [2 halves][PH_BYTES]
+  static constexpr int OFF_STAGE = OFF_SIDE;               // CTA 0: [2][PH_BYTES]
   static constexpr int OFF_ALPHA = OFF_SIDE;               // CTA 1: float [NPB][128]
-  static constexpr int OFF_L = OFF_ALPHA + NPB * TILE * 4; // CTA 1: float [SPLIT][128] partial sums
-  static constexpr int OFF_M = OFF_L + SPLIT * TILE * 4;   // CTA 1: float [128] row maxima (log2)
-  static constexpr int OFF_EV = OFF_STAGE + 2 * PH_BYTES;  // CTA 1: event {type, arg0, arg1, arg2}
+  static constexpr int OFF_L = OFF_ALPHA + NPB * TILE * 4; // CTA 1: float [2][128] row sums by half
+  static constexpr int OFF_M = OFF_L + 2 * TILE * 4;       // CTA 1: float [128] row maxima (log2)
+  static constexpr int OFF_EV = OFF_SIDE + 2 * PH_BYTES;  // CTA 1: event {type, arg0, arg1, arg2}
   static constexpr int OFF_FLAGS = OFF_EV + 16;            // int [4]: abort, tmem
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
   // full[3] empty[3] s_full[2] s_free[2] q_cp p_free[4] p_full[4] o_item
-  // o_sync ev_go ev_done l_full drain stage_free l_free (the same layout
+  // o_sync ev_go ev_done l_full drain stage_free[2] l_free (the same layout
   // in both CTAs: p_free is reached by a multicast commit, the others by
   // mapa)
-  static constexpr int NBAR = 2 * RING + 2 + 2 + 1 + 2 * NPB + 1 + 1 + 1 + 1 + 1 + 1 + 1 + 1;
-  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8;
+  static constexpr int NBAR = 2 * RING + 2 + 2 + 1 + 2 * NPB + 1 + 1 + 1 + 1 + 1 + 1 + 2 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int TMEM_S = 0;               // CTA 0: S buffers, 128 columns each
   static constexpr int TMEM_Q = 256;             // CTA 0: Q, 8 columns per 16-element K step
   static constexpr int TMEM_O = 0;               // CTA 1: O, 512 columns
@@ -115,21 +112,9 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  // The layout fills the shared memory limit with no alignment slack: a base
-  // that is not 1024-byte aligned (never seen: the dynamic window starts
-  // aligned) is reported instead of used.  Both CTAs see the same base and
-  // leave before any cluster barrier.
-  if (smem != smem_raw) {
-    if (threadIdx.x == 0) {
-      atomicCAS(&g_attn_error, 0u, 1u | (89u << 8));
-      atomicOr(&g_attn_error, 1u);
-    }
-    return;
-  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t ring = sbase + T::OFF_RING;
   const uint32_t pbuf = sbase + T::OFF_P;
-  float* xch = reinterpret_cast<float*>(smem + T::OFF_XCH);        // CTA 0
   const uint32_t stage = sbase + T::OFF_STAGE;                      // CTA 0
   float* alpha_sm = reinterpret_cast<float*>(smem + T::OFF_ALPHA);  // CTA 1
   float* l_sm = reinterpret_cast<float*>(smem + T::OFF_L);          // CTA 1
@@ -151,8 +136,8 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
   const uint32_t ev_done = ev_go + 8;                 // CTA 1: event handled
   const uint32_t l_full = ev_done + 8;                // CTA 1: row sums and maxima landed
   const uint32_t drain = l_full + 8;
-  const uint32_t stage_free = drain + 8;              // CTA 0: the staged tile has landed in CTA 1
-  const uint32_t l_free = stage_free + 8;             // CTA 0: CTA 1 has read the row sums
+  const uint32_t stage_free = drain + 8;              // [2] CTA 0: a staged P half has landed in CTA 1
+  const uint32_t l_free = stage_free + 16;            // CTA 0: CTA 1 has read the row sums
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -164,7 +149,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(s_free + 8 * i, T::WORK_WARPS);
+      mbar_init(s_free + 8 * i, T::SM_WARPS);
     }
     for (int i = 0; i < T::NPB; ++i) {
       mbar_init(p_free + 8 * i, 1);
@@ -178,6 +163,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     mbar_init(l_full, 1);
     mbar_init(drain, 1);
     mbar_init(stage_free, 1);
+    mbar_init(stage_free + 8, 1);
     mbar_init(l_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -423,19 +409,18 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     }
     post(AB_EV_STOP, 0, 0, 0);
     if (!ok) *abort_flag = 1;
-  } else if (cr == 0 && warp >= 2 && warp < T::RELAY_WARP) {
+  } else if (cr == 0 && warp >= 2 && warp < 2 + T::SM_WARPS) {
     // ---------------------------------------------------- CTA 0: softmax
-    // SPLIT threads per q row: warps with the same warp % 4 share a TMEM lane
-    // quarter; quarter-mate qd owns keys [KS qd, KS qd + KS) of each 64-key
-    // half tile.  The group meets on named barrier 1 + wq; a failed wait
-    // only clears `ok`, and the group leaves together after the next barrier
-    // that ANDs `ok` over it.
-    constexpr int KS = T::KS;
+    // Warp w reads TMEM lane quarter w % 4 (32 q rows) and owns 64-key half
+    // hh = (w - 2) / 4 of every tile.  Each thread takes its row's maximum
+    // over the whole tile itself (the two warps of a quarter do it twice
+    // rather than exchange it), then the weights of its half, written into
+    // the half's staging buffer and shipped by one 4 KB bulk copy per warp
+    // (its 32 rows are contiguous in the P layout).
     const int wq = warp & 3;
-    const int qd = (warp - 2) >> 2;
+    const int hh = (warp - 2) >> 2;
     const int row = wq * 32 + lane;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    auto group_and = [&](bool v) { return named_bar_and(1 + wq, 32 * T::SPLIT, v); };
     volatile int own_abort = 0;
     const uint32_t p_full_1 = mapa_shared(p_full, 1);
     const uint32_t pbuf_1 = mapa_shared(pbuf, 1);
@@ -443,155 +428,135 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     const uint32_t l_1 = mapa_shared(smem_u32(l_sm), 1);
     const uint32_t m_1 = mapa_shared(smem_u32(m_sm), 1);
     const uint32_t l_full_1 = mapa_shared(l_full, 1);
-    // this thread's two 16-byte units of a P half row, at the same offsets
-    // in a staging buffer and in CTA 1's P buffer (K-major, 128-byte
-    // swizzle: unit v of row r at 128 r + ((v ^ (r & 7)) * 16)); the 32 rows
-    // of a lane quarter are one contiguous 4 KB block
-    const uint32_t pofs0 = row * 128 + (((2 * qd) ^ (row & 7)) << 4);
-    const uint32_t pofs1 = row * 128 + (((2 * qd + 1) ^ (row & 7)) << 4);
-    static_assert(KS == 16, "two 16-byte units of P per thread and half");
-    bool ok = true;   // this warp's waits
-    bool gok = true;  // the group's, from its last barrier
-    int j = 0, h = 0, nitem = 0;
-    for (int L = item0; L < p.n_items; L += istride) {
+    // P half layout, the same in a staging buffer and in CTA 1's P buffers:
+    // K-major, 128-byte swizzle, 16-byte unit v of row r at 128 r + ((v ^
+    // (r & 7)) * 16)
+    const uint32_t sbuf = stage + hh * T::PH_BYTES + row * 128;
+    bool ok = true;
+    int j = 0, nitem = 0;
+    for (int L = item0; L < p.n_items && ok; L += istride) {
       const PrefillItem it = prefill_item(p, L, 0);
       if (it.ntiles == 0) continue;  // CTA 1 writes the empty item
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
       lim = max(0, min(it.skv, lim));
-      float m_used = -INFINITY;  // log2-domain running max, the same in the group
-      float l = 0.f;             // this thread's share of the row sum
-      for (int t = 0; t < it.ntiles; ++t, ++j) {
+      float m_used = -INFINITY;  // log2-domain running max
+      float la[4] = {0.f, 0.f, 0.f, 0.f};  // the half's row sum, in four independent parts
+      for (int t = 0; t < it.ntiles && ok; ++t, ++j) {
         const int sb = j & 1;
-        if (ok) ok = mbar_wait_warp(s_full + 8 * sb, (j >> 1) & 1, &own_abort, tmo, 83);
-        if (ok) tc_fence_after();
+        const int h = 2 * j + hh;   // P half index
+        const int pb = h % T::NPB;  // CTA 1's P buffer
+        const uint32_t srow = tmem + lane_base + T::TMEM_S + sb * 128;
+        ok = mbar_wait_warp(s_full + 8 * sb, (j >> 1) & 1, &own_abort, tmo, 83);
+        if (!ok) break;
+        tc_fence_after();
         const int tile0 = t * T::KT;
         const int win0 = min(tile0, it.skv - T::KT);
-        // both halves of this thread's slice of the tile: keys win0 + 64 hh +
-        // KS qd + e (a shifted last window's keys below tile0 belong to the
-        // previous tile)
-        float s[2 * KS];
-        float mx = -INFINITY;
         // a tile wholly inside [0, lim) for this row: no mask, and a quarter
-        // of its exponentials go to the FMA pipe
+        // of its exponentials go to the FMA pipe.  Column c of the tile is
+        // key win0 + c (a shifted last window's keys below tile0 belong to
+        // the previous tile).
         const bool whole = win0 == tile0 && tile0 + T::KT <= lim;
-        if (ok) {
-          tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + qd * KS, *reinterpret_cast<float(*)[16]>(s));
-          tmem_ld16(tmem + lane_base + T::TMEM_S + sb * 128 + T::HT + qd * KS,
-                    *reinterpret_cast<float(*)[16]>(s + KS));
+        // pass 1: the row maximum of the raw scores over the tile (scale > 0
+        // keeps the order); the next 32 columns load while these are folded
+        float mx = -INFINITY;
+        {
+          float v[2][32];
+          tmem_ld<32>(srow, v[0]);
           tmem_wait_ld();
-        }
-        // S buffer sb has been read: the next S may go there
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + 8 * sb);
-        if (ok) {
-          // raw scores here (scale > 0 keeps the order)
-          if (whole) {
 #pragma unroll
-            for (int e = 0; e < 2 * KS; e += 2) mx = fmaxf(mx, fmaxf(s[e], s[e + 1]));
-          } else {
+          for (int c = 0; c < 4; ++c) {
+            if (c < 3) tmem_ld<32>(srow + 32 * (c + 1), v[(c + 1) & 1]);
+            const float* w = v[c & 1];
+            if (whole) {
 #pragma unroll
-            for (int e = 0; e < 2 * KS; ++e) {
-              const int key = win0 + (e / KS) * T::HT + qd * KS + (e % KS);
-              s[e] = (key >= tile0 && key < lim) ? s[e] : -INFINITY;
-              mx = fmaxf(mx, s[e]);
+              for (int e = 0; e < 32; e += 2) mx = fmaxf(mx, fmaxf(w[e], w[e + 1]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int key = win0 + 32 * c + e;
+                if (key >= tile0 && key < lim) mx = fmaxf(mx, w[e]);
+              }
             }
+            if (c < 3) tmem_wait_ld();
           }
         }
-        // the row maximum over the tile's 128 keys.  One exchange buffer is
-        // enough: every thread has read it before it passes the barriers of
-        // this tile's halves, and it is written again only after them.
-        xch[qd * T::TILE + row] = mx;
-        gok = group_and(ok);
-        ok = gok;
-        if (!gok) break;
-        float tm = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < T::SPLIT; ++k) tm = fmaxf(tm, xch[k * T::TILE + row]);
-        tm *= p.scale_log2;
+        const float tm = mx * p.scale_log2;
         // lazy raise (threshold 8 in log2 units): the weights stay <= 256
         const bool need = tm > m_used + 8.f;
         const float mn = need ? tm : m_used;
         const float alpha = need ? ex2(m_used - mn) : 1.f;  // m_used = -inf: 0
         m_used = mn;
-        l *= alpha;
-        // an invisible key's weight is exactly 0 (ex2(-inf) = +0); a row
-        // with no visible key yet keeps m_used = -inf and all weights 0
+#pragma unroll
+        for (int k = 0; k < 4; ++k) la[k] *= alpha;
+        // an invisible key's weight is exactly 0; a row with no visible key
+        // yet keeps m_used = -inf and all weights 0
         const float neg_mu = m_used == -INFINITY ? 0.f : -m_used;
-        // both halves' P, then one staging write, one barrier and the
-        // copies of the whole tile
-        uint32_t u[2][KS / 2];
-        if (whole) {
+        // pass 2: this half's weights.  The staging buffer last held the
+        // previous tile's half: CTA 1 reports when it landed.
+        if (j >= 1) ok = mbar_wait_warp(stage_free + 8 * hh, (j - 1) & 1, &own_abort, tmo, 91);
+        if (!ok) break;
+        {
+          float v[2][32];
+          tmem_ld<32>(srow + hh * T::HT, v[0]);
+          tmem_ld<32>(srow + hh * T::HT + 32, v[1]);
+          tmem_wait_ld();
+          // S buffer sb has been read by this warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + 8 * sb);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
+          for (int c = 0; c < 2; ++c) {
+            uint32_t u[16];
+            if (whole) {
 #pragma unroll
-            for (int e = 0; e < KS; e += 2) {
-              const float p0 = ex2(fmaf(s[hh * KS + e], p.scale_log2, neg_mu));
-              const float x1 = fmaf(s[hh * KS + e + 1], p.scale_log2, neg_mu);
-              const float p1 = (e & 2) ? ex2_fma(x1) : ex2(x1);
-              l += p0 + p1;
-              u[hh][e / 2] = pack2(p0, p1, BF16);
-            }
-        } else {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int e = 0; e < KS; e += 2) {
-              const float p0 = ex2(fmaf(s[hh * KS + e], p.scale_log2, neg_mu));
-              const float p1 = ex2(fmaf(s[hh * KS + e + 1], p.scale_log2, neg_mu));
-              l += p0 + p1;
-              u[hh][e / 2] = pack2(p0, p1, BF16);
-            }
-        }
-        // the staging buffer last held tile j - 1: CTA 1 reports once it has
-        // seen both of its halves land
-        if (ok && j >= 1) ok = mbar_wait_warp(stage_free, (j - 1) & 1, &own_abort, tmo, 91);
-        if (ok) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            st_shared_v4(stage + hh * T::PH_BYTES + pofs0, u[hh][0], u[hh][1], u[hh][2], u[hh][3]);
-            st_shared_v4(stage + hh * T::PH_BYTES + pofs1, u[hh][4], u[hh][5], u[hh][6], u[hh][7]);
-          }
-          fence_proxy_async_smem();  // for the bulk copies' reads
-        }
-        gok = group_and(ok);
-        ok = gok;
-        if (!gok) break;
-        // The quarter's two copies and the rescale factors of the tile's
-        // first half, one job per warp of the group: qd = 0 copies half 0,
-        // qd = 1 half 1, qd = 2 sends the factors.  CTA 1's P buffer pb +
-        // hh was last read by PV(h + hh - NPB).  A failed wait here reaches
-        // the group at its next barrier.
-        const int pb = h % T::NPB;  // h is even, NPB too: pb + 1 is the next buffer
-        if (qd < 3) {
-          const int hh = qd & 1;
-          if (ok && h >= T::NPB)
-            ok = mbar_wait_warp_cluster(p_free + 8 * (pb + hh), ((h / T::NPB) - 1) & 1, &own_abort, tmo, 84);
-          if (ok) {
-            const uint32_t bar = p_full_1 + 8 * (pb + hh);
-            if (qd < 2) {
-              if (lane == 0)
-                bulk_copy_to_peer(pbuf_1 + (pb + hh) * T::PH_BYTES + wq * T::PQ_BYTES,
-                                  stage + hh * T::PH_BYTES + wq * T::PQ_BYTES, T::PQ_BYTES, bar);
+              for (int e = 0; e < 32; e += 2) {
+                const float p0 = ex2(fmaf(v[c][e], p.scale_log2, neg_mu));
+                const float x1 = fmaf(v[c][e + 1], p.scale_log2, neg_mu);
+                const float p1 = (e & 2) ? ex2_fma(x1) : ex2(x1);
+                la[(e >> 1) & 3] += p0 + p1;
+                u[e / 2] = pack2(p0, p1, BF16);
+              }
             } else {
-              // O's rescale factor before the tile's first PV
-              st_async_f32(alpha_1 + (pb * T::TILE + row) * 4, alpha, bar);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const int key = win0 + hh * T::HT + 32 * c + e;
+                const float p0 = (key >= tile0 && key < lim) ? ex2(fmaf(v[c][e], p.scale_log2, neg_mu)) : 0.f;
+                const float p1 =
+                    (key + 1 >= tile0 && key + 1 < lim) ? ex2(fmaf(v[c][e + 1], p.scale_log2, neg_mu)) : 0.f;
+                la[(e >> 1) & 3] += p0 + p1;
+                u[e / 2] = pack2(p0, p1, BF16);
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int unit = 4 * c + k;  // 8 keys per 16-byte unit
+              st_shared_v4(sbuf + ((unit ^ (row & 7)) << 4), u[4 * k], u[4 * k + 1], u[4 * k + 2],
+                           u[4 * k + 3]);
             }
           }
         }
-        h += 2;
+        fence_proxy_async_smem();  // for the bulk copy's reads
+        // CTA 1's P buffer pb and its rescale factors were last read by PV(h - NPB)
+        if (h >= T::NPB)
+          ok = mbar_wait_warp_cluster(p_free + 8 * pb, ((h / T::NPB) - 1) & 1, &own_abort, tmo, 84);
+        __syncwarp();  // every lane's row is staged
+        if (!ok) break;
+        const uint32_t bar = p_full_1 + 8 * pb;
+        if (lane == 0)
+          bulk_copy_to_peer(pbuf_1 + pb * T::PH_BYTES + wq * T::PQ_BYTES,
+                            stage + hh * T::PH_BYTES + wq * T::PQ_BYTES, T::PQ_BYTES, bar);
+        // O's rescale factor before the tile's first PV
+        if (hh == 0) st_async_f32(alpha_1 + (pb * T::TILE + row) * 4, alpha, bar);
       }
-      if (!gok) break;  // the same in the whole group (set by its last barrier)
-      // the partial row sums and the row maximum, once CTA 1 has read the
-      // previous item's.  A failed wait only clears `ok`: the group learns
-      // of it at its next barrier.
-      if (ok && nitem > 0) ok = mbar_wait_warp_cluster(l_free, (nitem - 1) & 1, &own_abort, tmo, 92);
+      if (!ok) break;
+      // the half's row sum (and the row maximum), once CTA 1 has read the
+      // previous item's
+      if (nitem > 0) ok = mbar_wait_warp_cluster(l_free, (nitem - 1) & 1, &own_abort, tmo, 92);
+      if (!ok) break;
       ++nitem;
-      if (ok) {
-        st_async_f32(l_1 + (qd * T::TILE + row) * 4, l, l_full_1);
-        if (qd == 0) st_async_f32(m_1 + row * 4, m_used, l_full_1);
-      }
+      st_async_f32(l_1 + (hh * T::TILE + row) * 4, (la[0] + la[1]) + (la[2] + la[3]), l_full_1);
+      if (hh == 0) st_async_f32(m_1 + row * 4, m_used, l_full_1);
     }
     if (!ok) *abort_flag = 1;
   } else if (cr == 1 && warp >= 2 && warp < T::RELAY_WARP) {
@@ -644,9 +609,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
                mbar_wait_warp_cluster(l_full, nl & 1, &own_abort, tmo, 87);
           if (ok) {
             tc_fence_after();
-            float lt = 0.f;  // the row sum from the scores CTA's SPLIT shares
-#pragma unroll
-            for (int k = 0; k < T::SPLIT; ++k) lt += l_sm[k * T::TILE + row];
+            const float lt = l_sm[row] + l_sm[T::TILE + row];
             inv = lt > 0.f ? 1.f / lt : 0.f;
             if (lt > 0.f) lse = (m_sm[row] + __log2f(lt)) * 0.69314718055994531f;
           }
@@ -695,21 +658,19 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     if (!ok) *abort_flag = 1;
   } else if (cr == 1 && warp == T::RELAY_WARP) {
     // ---------------------------------------------------- CTA 1: P arrivals -> CTA 0
-    // Watches the P buffers fill, in order, and tells CTA 0 as soon as both
-    // halves of a tile have landed, so that its staging buffer can take the
-    // next tile.  (The MMA issuer waits on the same barriers; a phase cannot
-    // complete twice before this warp sees it, since the copies that would
-    // complete it next come from a staging buffer this warp must free first.)
+    // Watches the P buffers fill, in order, and tells CTA 0 as soon as a
+    // half has landed, so that its staging buffer can take the next one.
+    // (The MMA issuer waits on the same barriers; a phase cannot complete
+    // twice before this warp sees it, since the copies that would complete
+    // it next come from a staging buffer this warp must free first.)
     const uint32_t stage_free_0 = mapa_shared(stage_free, 0);
     bool ok = true;
     int h = 0;
     for (int L = item0; L < p.n_items && ok; L += istride) {
       const PrefillItem it = prefill_item(p, L, 0);
-      for (int t = 0; t < it.ntiles && ok; ++t, h += 2) {
-        ok = mbar_wait_warp_cluster(p_full + 8 * (h % T::NPB), (h / T::NPB) & 1, abort_flag, tmo, 93) &&
-             mbar_wait_warp_cluster(p_full + 8 * ((h + 1) % T::NPB), ((h + 1) / T::NPB) & 1, abort_flag,
-                                    tmo, 93);
-        if (ok && lane == 0) mbar_arrive_remote_relaxed(stage_free_0);
+      for (int hh = 0; hh < 2 * it.ntiles && ok; ++hh, ++h) {
+        ok = mbar_wait_warp_cluster(p_full + 8 * (h % T::NPB), (h / T::NPB) & 1, abort_flag, tmo, 93);
+        if (ok && lane == 0) mbar_arrive_remote_relaxed(stage_free_0 + 8 * (h & 1));
         __syncwarp();
       }
     }
