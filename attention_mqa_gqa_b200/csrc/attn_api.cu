@@ -358,32 +358,13 @@ attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, cons
   return ATTN_OK;
 }
 
-template <int DK, int DVH, bool BF16, bool PAIR = false>
+template <int DK, int DVH, bool BF16>
 attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                              const attn::PrefillParams& pp, const attn_plan_t& pl,
                              cudaStream_t st) {
-  using Tr = attn::PrefillTraits<DK, DVH, PAIR>;
-  auto kern = attn::prefill_kernel<DK, DVH, BF16, PAIR>;
+  using Tr = attn::PrefillTraits<DK, DVH>;
+  auto kern = attn::prefill_kernel<DK, DVH, BF16>;
   set_smem(kern, Tr::SMEM_BYTES);
-  if constexpr (PAIR) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
-    cfg.blockDim = dim3(Tr::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, pp) != cudaSuccess) {
-      cudaGetLastError();
-      return ATTN_ECUDA;
-    }
-    return ATTN_OK;
-  }
   kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   return ATTN_OK;
@@ -553,7 +534,6 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
   pp.Sq = Sq;
   pp.n_qtiles = (Sq + 127) / 128;
   pp.dv_parts = pl.dv_parts;
-  pp.pairs = 0;
   pp.n_items = pp.n_qtiles * Hq * B * pl.dv_parts;  // per CTA, or per pair (split matmuls)
   {
     // K/V bytes of one kv head over the batch; blocks of kv heads whose

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
       if (++grp == T::RING) { grp = 0; ph ^= 1u; }
     };
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) continue;
       load(&tmQ, it.q0, 0, it.h, it.b, pol_q);
       load(&tmQ, it.q0, 4, it.h, it.b, pol_q);
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     uint32_t ph = 0;
     bool ok = true;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       for (int t = 0; t < it.ntiles && ok; ++t) {
         const int win0 = min(t * T::KT, it.skv - T::KT);
         for (int hh = 0; hh < 2 && ok; ++hh) {
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     bool ok = true;
     int j = 0, kq = 0;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) continue;
       // the previous item's S UMMAs read TMEM Q: wait for the last of them
       if (j > 0) ok = mbar_wait_warp(s_full + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, tmo, 72);
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
       ++ne;
     };
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) {
         post(AB_EV_EMPTY, L, 0, 0);
         continue;
@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     bool ok = true;
     int j = 0, nitem = 0;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) continue;  // CTA 1 writes the empty item
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
         }
         tc_fence_before();
       } else {  // AB_EV_OUTPUT, AB_EV_EMPTY: O / l -> out for item a0
-        const PrefillItem it = prefill_item(p, a0, 0);
+        const PrefillItem it = prefill_item(p, a0);
         const int qi = it.q0 + row;
         float inv = 0.f, lse = -INFINITY;
         if (type == AB_EV_OUTPUT) {
@@ -667,7 +667,7 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
     bool ok = true;
     int h = 0;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, 0);
+      const PrefillItem it = prefill_item(p, L);
       for (int hh = 0; hh < 2 * it.ntiles && ok; ++hh, ++h) {
         ok = mbar_wait_warp_cluster(p_full + 8 * (h % T::NPB), (h / T::NPB) & 1, abort_flag, tmo, 93);
         if (ok && lane == 0) mbar_arrive_remote_relaxed(stage_free_0 + 8 * (h & 1));

@@ -18,11 +18,10 @@
 // shared-memory bandwidth; the S buffer is reused for tile j + 2 once PV(j)
 // has completed.
 //
-// TMEM holds 512 fp32 columns per SM.  Two S buffers (256 columns) plus a
-// 128 x 512 fp32 O would need 768, so at d_v = 512 two work items share a
-// q tile, each owning half of d_v (DVH = 256) and each recomputing S.  The
-// K/V tiles those items (and the G heads of the group) read are the same,
-// so they come from L2.
+// TMEM holds 512 fp32 columns per SM: two S buffers (256 columns) and O
+// (DVH = 128 columns).  (At d_k = d_v = 512 a 128 x 512 fp32 O alone fills
+// TMEM; that case runs on SM pairs that split the two matmuls, in
+// prefill_ab_kernel.cuh.)
 //
 // The grid is persistent: one CTA per SM walks the work items in
 // heavy-first order (the last q tiles see the most keys under the causal
@@ -31,8 +30,8 @@
 //
 // Warp roles: warp 0 lane 0 streams K/V chunks through a ring of 32 KB
 // groups and lane 1 loads Q per item (TMA), warp 1 allocates TMEM and issues
-// UMMA, the other warps (8 at d_k = 512, else 16) run the softmax, rescale
-// and epilogue: SPLIT threads per q row (warps with the same index mod 4
+// UMMA, the other 16 warps run the softmax, rescale and epilogue: SPLIT
+// threads per q row (warps with the same index mod 4
 // share a TMEM lane quarter), each owning a slice of the row's keys and of
 // its output columns, exchanging the row maximum and sum through shared
 // memory.
@@ -50,7 +49,6 @@ struct PrefillParams {
   int B, Hq, Hkv, G, Sq;
   int n_qtiles, dv_parts, n_items;
   int heads_per_block;        // q heads (a multiple of G) whose items run together
-  int pairs;                  // 1: a cluster of two CTAs takes two heads of one kv group
   float scale_log2;           // scale * log2(e), scale > 0
   int causal;
   uint64_t timeout_ns;
@@ -66,12 +64,9 @@ struct PrefillItem {
 // block the heaviest q tiles come first, and the dv parts and heads of one
 // q tile are adjacent so that CTAs running at the same time read the same
 // K/V tiles.
-// With pairs, "heads" below are head pairs (2u, 2u + 1) and CTA `cr` of the
-// pair takes head 2u + cr.
-__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int L, int cr = 0) {
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int L) {
   PrefillItem it;
-  const int U = p.pairs ? 2 : 1;
-  const int units = p.Hq / U, units_per_block = p.heads_per_block / U;
+  const int units = p.Hq, units_per_block = p.heads_per_block;
   const int per_head = p.n_qtiles * p.B * p.dv_parts;
   const int blk = L / (units_per_block * per_head);
   L -= blk * units_per_block * per_head;
@@ -79,7 +74,7 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   const int nh = min(units_per_block, units - h0);  // head units of this block
   it.part = L % p.dv_parts;
   L /= p.dv_parts;
-  it.h = (h0 + L % nh) * U + cr;
+  it.h = h0 + L % nh;
   L /= nh;
   it.b = L % p.B;
   const int qt = p.n_qtiles - 1 - L / p.B;
@@ -93,11 +88,7 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
   return it;
 }
 
-// PAIR: clusters of two CTAs on two SMs run the MMAs as one (cta_group::2):
-// M = 256 = the two CTAs' q tiles (two heads of one kv group, same rows),
-// and the B operands are split between them -- each CTA copies 64 of a K
-// tile's 128 keys and 128 of V's DVH = 256 columns, half the per-SM copies.
-template <int DK, int DVH, bool PAIR = false>
+template <int DK, int DVH>
 struct PrefillTraits {
   static constexpr int TILE = 128;               // q rows per item (MMA M)
   static constexpr int KT = 128;                 // keys per tile (MMA N of S)
@@ -106,12 +97,10 @@ struct PrefillTraits {
                                                  // last one zero-filled if KCH is odd
   static constexpr int VCH = DVH / 64;           // V chunks per key tile (this item's columns)
   // softmax threads per q row: 4 (the softmax is bound by instruction
-  // issue: more warps hide more latency), except 2 at d_k = 512 on one SM,
-  // where shared memory has no room for the larger exchange buffers
-  static constexpr int SPLIT = (DK >= 512 && !PAIR) ? 2 : 4;
-  static constexpr int NQ = (DK >= 512 || QCH > 2) ? 1 : 2;  // Q buffers
-  // 16 KB chunk slots (pairs copy half as much per SM: a shallower ring)
-  static constexpr int RING = PAIR ? 4 : (DK >= 512 ? 6 : 8);
+  // issue: more warps hide more latency)
+  static constexpr int SPLIT = 4;
+  static constexpr int NQ = QCH > 2 ? 1 : 2;     // Q buffers
+  static constexpr int RING = 8;                 // 16 KB chunk slots
   static constexpr int SLOT = 16384;
   // one TMA copy moves GCH consecutive 64-column chunks (one ring group):
   // copies of a single 16 KB chunk cap a CTA's stream well below what the
@@ -123,9 +112,8 @@ struct PrefillTraits {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + NQ * Q_BYTES;
   // row exchange buffers float [XR][SPLIT][128]: two rounds alternate with
-  // the tile (one barrier per exchange); at d_k = 512 shared memory has room
-  // for one round only, which then takes a second barrier
-  static constexpr int XR = (DK >= 512 && !PAIR) ? 1 : 2;
+  // the tile (one barrier per exchange)
+  static constexpr int XR = 2;
   static constexpr int OFF_XCH = OFF_RING + RING * SLOT;
   static constexpr int OFF_FLAGS = OFF_XCH + XR * SPLIT * 128 * 4;  // abort, tmem base
   static constexpr int OFF_BAR = OFF_FLAGS + 16;
@@ -139,24 +127,19 @@ struct PrefillTraits {
                                                  // overwrites the first 64 of S(j)
   static constexpr int TMEM_O = 256;             // DVH columns
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int K_ROWS = PAIR ? 64 : 128;      // K rows this CTA copies per tile
-  static constexpr int K_GCH = PAIR ? 4 : GCH;        // K chunks per copy (32 KB)
-  static constexpr int V_CH = PAIR ? 2 : VCH;         // V chunks this CTA copies per tile
-  static_assert(!PAIR || (DK == 512 && DVH == 256), "pairs: d = 512 prefill");
   static_assert(VCH % GCH == 0 && QCH % GCH == 0 && RING % GCH == 0 && GCH == 2,
                 "chunks travel in pairs; a V pair is one 128-column block of O");
   static_assert(TMEM_O + DVH <= 512, "TMEM");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int DK, int DVH, bool BF16, bool PAIR = false>
-__global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
+template <int DK, int DVH, bool BF16>
+__global__ void __launch_bounds__(PrefillTraits<DK, DVH>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using T = PrefillTraits<DK, DVH, PAIR>;
-  const uint32_t cr = PAIR ? cluster_ctarank() : 0u;  // PAIR: 0 issues the pair MMAs
-  const int item0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int istride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  using T = PrefillTraits<DK, DVH>;
+  const int item0 = (int)blockIdx.x;
+  const int istride = (int)gridDim.x;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -192,35 +175,27 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + 8 * i, 1);
-      mbar_init(p_full + 8 * i, (PAIR ? 2 : 1) * T::SOFTMAX_THREADS);
+      mbar_init(p_full + 8 * i, T::SOFTMAX_THREADS);
       mbar_init(o_done + 8 * i, 1);
     }
-    mbar_init(o_free, (PAIR ? 2 : 1) * T::SOFTMAX_THREADS);
+    mbar_init(o_free, T::SOFTMAX_THREADS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(smem_u32(tmem_slot), T::TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
-  if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // waits on phases that the other CTA of a pair may complete use cluster scope
   auto wait1 = [&](uint32_t bar, uint32_t parity, volatile int* ab, uint32_t id) {
-    return PAIR ? mbar_wait_cluster(bar, parity, ab, p.timeout_ns, id)
-                : mbar_wait(bar, parity, ab, p.timeout_ns, id);
+    return mbar_wait(bar, parity, ab, p.timeout_ns, id);
   };
   auto waitw = [&](uint32_t bar, uint32_t parity, volatile int* ab, uint32_t id) {
-    return PAIR ? mbar_wait_warp_cluster(bar, parity, ab, p.timeout_ns, id)
-                : mbar_wait_warp(bar, parity, ab, p.timeout_ns, id);
+    return mbar_wait_warp(bar, parity, ab, p.timeout_ns, id);
   };
 
   if (warp == 0 && lane == 0) {
@@ -231,22 +206,14 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     int grp = 0;
     uint32_t ph = 0;
     bool ok = true;
-    // chunks [ch, ch + GCH) of key rows [row, row + 128) -> the next ring group
-    // one copy (32 KB) starting at chunk `ch` of rows `row`.. -> the next
-    // ring group; with pairs the bytes of both CTAs' copies are counted on
-    // CTA 0's barrier
+    // one copy (32 KB) of chunks [ch, ch + GCH) of key rows [row, row +
+    // 128) -> the next ring group
     auto load = [&](const CUtensorMap* map, int ch, int row, int kvh, int b) {
       if (!ok) return;
       ok = wait1(empty_bar(grp), ph ^ 1u, abort_flag, 21);
       if (!ok) return;
-      if constexpr (PAIR) {
-        if (cr == 0) mbar_arrive_expect_tx(full_bar(grp), 2 * T::GBYTES);
-        tma_load_5d_pair(ring + grp * T::GBYTES, map, mapa_shared(full_bar(grp), 0), 0, row, ch,
-                         kvh, b, pol_kv);
-      } else {
-        mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
-        tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, row, ch, kvh, b, pol_kv);
-      }
+      mbar_arrive_expect_tx(full_bar(grp), T::GBYTES);
+      tma_load_5d(ring + grp * T::GBYTES, map, full_bar(grp), 0, row, ch, kvh, b, pol_kv);
       if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
     };
     bool have_prev = false;
@@ -256,21 +223,19 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     // past skv -- possibly unwritten memory -- enters P.V; a negative start
     // reads zeros.
     auto load_v = [&]() {
-      for (int c = 0; c < T::V_CH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
+      for (int c = 0; c < T::VCH; c += T::GCH) load(&tmV, pv_ch + c, pv_tok, pv_kvh, pv_b);
     };
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, (int)cr);
+      const PrefillItem it = prefill_item(p, L);
       for (int j = 0; j < it.ntiles && ok; ++j) {
         if (j == 0 && have_prev) load_v();  // finish the previous item first
         const int row0 = min(j * T::KT, it.skv - T::KT);
-        for (int c = 0; c < T::KCH; c += T::K_GCH)
-          load(&tmK, c, row0 + (int)cr * T::K_ROWS, it.kvh, it.b);
+        for (int c = 0; c < T::KCH; c += T::GCH) load(&tmK, c, row0, it.kvh, it.b);
         if (j > 0) load_v();
         pv_tok = row0;
         pv_kvh = it.kvh;
         pv_b = it.b;
-        // pairs: this CTA's half of the part's DVH columns
-        pv_ch = it.part * (DVH / 64) + (int)cr * T::V_CH;
+        pv_ch = it.part * (DVH / 64);
         have_prev = true;
       }
     }
@@ -282,41 +247,30 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     int kq = 0;
     bool ok = true;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, (int)cr);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) continue;
       const int qb = kq % T::NQ;
       if (kq >= T::NQ)  // buffer qb was last read by the S MMAs of item kq - NQ
         ok = wait1(q_free + 8 * qb, ((kq - T::NQ) / T::NQ) & 1, abort_flag, 22);
       if (!ok) break;
-      if constexpr (PAIR) {
-        if (cr == 0) mbar_arrive_expect_tx(q_full + 8 * qb, 2 * T::Q_BYTES);
-        const uint32_t lead = mapa_shared(q_full + 8 * qb, 0);
-        for (int c = 0; c < T::QCH; c += T::GCH)
-          tma_load_5d_pair(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, lead, 0, it.q0, c, it.h,
-                           it.b, pol_q);
-      } else {
-        mbar_arrive_expect_tx(q_full + 8 * qb, T::Q_BYTES);
-        for (int c = 0; c < T::QCH; c += T::GCH)
-          tma_load_5d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, 0, it.q0, c,
-                      it.h, it.b, pol_q);
-      }
+      mbar_arrive_expect_tx(q_full + 8 * qb, T::Q_BYTES);
+      for (int c = 0; c < T::QCH; c += T::GCH)
+        tma_load_5d(qs + qb * T::Q_BYTES + c * T::SLOT, &tmQ, q_full + 8 * qb, 0, it.q0, c, it.h,
+                    it.b, pol_q);
       ++kq;
     }
-  } else if (warp == 1 && (!PAIR || cr == 0)) {
+  } else if (warp == 1) {
     // ---------------------------------------------------- MMA issuer (whole warp,
     // one elected lane issues; waits are polled by the converged warp)
-    constexpr int M = PAIR ? 256 : 128;                                   // pairs: both q tiles
-    constexpr uint32_t idS = umma_idesc(M, 128, BF16, false, false);      // Q, K both K-major
-    constexpr uint32_t idO = umma_idesc(M, PAIR ? 256 : 128, BF16, false, true);  // P K, V MN-major
+    constexpr uint32_t idS = umma_idesc(128, 128, BF16, false, false);  // Q, K both K-major
+    constexpr uint32_t idO = umma_idesc(128, 128, BF16, false, true);   // P K, V MN-major
     auto mma_ss = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-      if constexpr (PAIR) umma_ss_pair(d, a, b, id, acc); else umma_ss(d, a, b, id, acc);
+      umma_ss(d, a, b, id, acc);
     };
     auto mma_ts = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
-      if constexpr (PAIR) umma_ts_pair(d, a, b, id, acc); else umma_ts(d, a, b, id, acc);
+      umma_ts(d, a, b, id, acc);
     };
-    auto commit = [&](uint32_t bar) {
-      if constexpr (PAIR) umma_commit_pair(bar); else umma_commit(bar);
-    };
+    auto commit = [&](uint32_t bar) { umma_commit(bar); };
     int grp = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -330,7 +284,7 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
       if (!ok) return;
       tc_fence_after();
       const uint32_t pcol = tmem + T::TMEM_S + pb * 128;  // P(t): 8 columns per 16 keys
-      for (int i = 0; i < T::V_CH / 2; ++i) {  // pairs: one group, N = 256 across the pair
+      for (int i = 0; i < T::VCH / 2; ++i) {  // one ring group = 128 columns of V
         ok = waitw(full_bar(grp), ph, abort_flag, 25);
         if (!ok) return;
         tc_fence_after();
@@ -356,7 +310,7 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     int j = 0, kq = 0, prev_k = 0;
     bool prev_first = false;
     for (int L = item0; L < p.n_items && ok; L += istride) {
-      const PrefillItem it = prefill_item(p, L, (int)cr);
+      const PrefillItem it = prefill_item(p, L);
       if (it.ntiles == 0) continue;
       const int qb = kq % T::NQ;
       for (int i = 0; i < it.ntiles && ok; ++i, ++j) {
@@ -370,25 +324,24 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
         if (j >= 2) ok = waitw(o_done + 8 * sb, ((j - 2) >> 1) & 1, abort_flag, 27);
         if (!ok) break;
         tc_fence_after();
-        for (int c = 0; c < T::KCH && ok; c += T::K_GCH) {
+        for (int c = 0; c < T::KCH && ok; c += T::GCH) {
           ok = waitw(full_bar(grp), ph, abort_flag, 28);
           if (!ok) break;
           tc_fence_after();
           if (elect_one()) {
             // A = Q chunks c.., B = the group's K chunks: both K-major, 128-byte
-            // swizzle, 8-row groups 1024 bytes apart, 32 bytes per K step.  A
-            // K chunk of the group is K_ROWS x 128 bytes (pairs: this CTA's 64
-            // of the tile's 128 keys, the pair MMA taking N = 128 from both).
+            // swizzle, 8-row groups 1024 bytes apart, 32 bytes per K step; a K
+            // chunk of the group is 128 keys x 128 bytes.
             const uint64_t ad0 = umma_sdesc(qs + qb * T::Q_BYTES + c * T::SLOT, 16, 1024, SMEM_SW128);
             const uint64_t bd0 = umma_sdesc(ring + grp * T::GBYTES, 16, 1024, SMEM_SW128);
             const uint32_t d = tmem + T::TMEM_S + sb * 128;
             mma_ss(d, ad0, bd0, idS, c > 0 ? 1u : 0u);
             // the second chunk of an odd count's last pair is padding: skipped
-            const int nks = c + T::K_GCH <= T::KCH ? 4 * T::K_GCH : 4 * (T::KCH - c);
+            const int nks = c + T::GCH <= T::KCH ? 4 * T::GCH : 4 * (T::KCH - c);
 #pragma unroll
-            for (int ks = 1; ks < 4 * T::K_GCH; ++ks) {
+            for (int ks = 1; ks < 4 * T::GCH; ++ks) {
               const uint64_t aoff = (uint64_t)((ks >> 2) * (T::SLOT >> 4) + (ks & 3) * 2);
-              const uint64_t boff = (uint64_t)((ks >> 2) * (T::K_ROWS * 128 >> 4) + (ks & 3) * 2);
+              const uint64_t boff = (uint64_t)((ks >> 2) * (T::KT * 128 >> 4) + (ks & 3) * 2);
               if (ks < nks) mma_ss(d, ad0 + aoff, bd0 + boff, idS, 1u);
             }
             commit(empty_bar(grp));
@@ -431,22 +384,13 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     auto wait = [&](uint32_t bar, uint32_t parity, uint32_t id) {
       return waitw(bar, parity, &own_abort, id);
     };
-    // pairs: the P and O handshakes are counted on CTA 0's barriers.  The
-    // thread's TMEM stores or reads have completed (tcgen05 wait + fence)
-    // before it arrives; CTA 1 arrives with a CTA-scope release, since a
-    // cluster-scope release stalls the thread while the SM streams copies.
-    auto arrive_lead = [&](uint32_t bar) {
-      if constexpr (PAIR) {
-        if (cr == 0) mbar_arrive(bar);
-        else mbar_arrive_remote_cta(mapa_shared(bar, 0));
-      } else {
-        mbar_arrive(bar);
-      }
-    };
+    // The thread's TMEM stores or reads have completed (tcgen05 wait +
+    // fence) before it arrives.
+    auto arrive_lead = [&](uint32_t bar) { mbar_arrive(bar); };
     bool ok = true;
     int j = 0;
     for (int L = item0; L < p.n_items; L += istride) {
-      const PrefillItem it = prefill_item(p, L, (int)cr);
+      const PrefillItem it = prefill_item(p, L);
       const int qi = it.q0 + row;
       int lim = p.causal ? qi + it.skv - p.Sq + 1 : it.skv;  // keys [0, lim) visible
       lim = max(0, min(it.skv, lim));
@@ -493,7 +437,6 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
         if (!ok) break;
 #pragma unroll
         for (int k = 0; k < SPLIT; ++k) mx = fmaxf(mx, xb[k * 128 + row]);
-        if (T::XR == 1) named_bar_sync(1 + wq, 32 * SPLIT);  // all have read the round
         mx *= p.scale_log2;
         // Raise the running max only when the tile's exceeds it by more than 8
         // (log2 units); weights stay <= 256 and O/l is unaffected.
@@ -562,7 +505,6 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
       float ltot = 0.f;
 #pragma unroll
       for (int k = 0; k < SPLIT; ++k) ltot += xb[k * 128 + row];
-      if (T::XR == 1) named_bar_sync(1 + wq, 32 * SPLIT);
       if (it.ntiles > 0) {
         const int t = j - 1;
         ok = wait(o_done + 8 * (t & 1), (t >> 1) & 1, 33);
@@ -602,37 +544,12 @@ __global__ void __launch_bounds__(PrefillTraits<DK, DVH, PAIR>::THREADS, 1)
     }
     if (!ok) *abort_flag = 1;
   }
-  if constexpr (PAIR) {
-    // After a give-up in either CTA, CTA 0's issued pair MMAs (reading both
-    // CTAs' shared memory and TMEM) and each CTA's copies must land before
-    // the pair leaves.
-    __syncthreads();
-    if (*abort_flag) {
-      if (warp == 1 && cr == 0) {
-        if (elect_one()) umma_commit_pair(drain);
-        __syncwarp();
-        volatile int never = 0;
-        mbar_wait_warp(drain, 0, &never, 1000000ull, 29);
-      }
-      if (threadIdx.x == 0) {
-        const uint64_t t0n = global_timer_ns();
-        while (global_timer_ns() - t0n < 2000000ull) __nanosleep(1000);
-      }
-    }
-    tc_fence_before();
-    cluster_sync_all();
-    if (warp == 1) {
-      tc_fence_after();
-      tmem_dealloc_pair(tmem, T::TMEM_COLS);
-    }
-  } else {
-    abort_tail(abort_flag, warp, drain);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-      tc_fence_after();
-      tmem_dealloc(tmem, T::TMEM_COLS);
-    }
+  abort_tail(abort_flag, warp, drain);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T::TMEM_COLS);
   }
 }
 

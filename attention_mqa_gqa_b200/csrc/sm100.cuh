@@ -513,25 +513,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(raddr), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_f32(uint32_t raddr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(raddr), "f"(v) : "memory");
-}
-
-// Arrive on an mbarrier in another CTA of the cluster (release at cluster
-// scope: this thread's earlier shared-memory writes, local or remote, are
-// visible to whoever acquires the phase).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
-               : "memory");
-}
-
 // Arrive on an mbarrier in another CTA of the cluster, relaxed: a signal
 // that carries no data (e.g. "this CTA has finished reading a buffer").  A
 // release at cluster scope stalls the arriving thread for about a
@@ -632,12 +613,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
-// Generic-proxy shared-memory writes (local or to the other CTA) made
-// visible to the async proxy (the pair's UMMA operand reads).
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
-
 // All threads of both CTAs (unbounded hardware barrier: only used where
 // every thread of the pair is known to arrive).
 __device__ __forceinline__ void cluster_sync_all() {
@@ -668,17 +643,6 @@ __device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t adesc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Pair UMMA with A read from each CTA's TMEM (its 128 rows).
-__device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

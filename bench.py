@@ -56,6 +56,8 @@ KERNEL_SOURCES = {
     "mla_pair_kernel": [_CSRC + "sm100.cuh", _CSRC + "decode_kernel.cuh", _CSRC + "mla_pair_kernel.cuh",
                         _CSRC + "attn_api.cu"],
     "prefill_kernel": [_CSRC + "sm100.cuh", _CSRC + "prefill_kernel.cuh", _CSRC + "attn_api.cu"],
+    "prefill_ab_kernel": [_CSRC + "sm100.cuh", _CSRC + "prefill_kernel.cuh", _CSRC + "prefill_ab_kernel.cuh",
+                          _CSRC + "attn_api.cu"],
     "gather_rows_kernel": [_CSRC + "sm100.cuh", _CSRC + "gather_rows.cuh", _CSRC + "attn_api.cu"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -626,7 +628,8 @@ def step_dist_of(g, steps):
 
 def kernel_name(w, g):
     if not g.decode:
-        return "prefill_kernel"
+        # d_k = 512: SM pairs that split the two matmuls
+        return "prefill_ab_kernel" if w.d_k == 512 else "prefill_kernel"
     return "mla_pair_kernel" if w.mla else "decode_split_kernel"
 
 
