@@ -44,7 +44,7 @@ class AttnError(RuntimeError):
 EXPORTS = ("attn_plan", "attn_workspace_bytes", "attn_fwd", "attn_decode_partial",
            "attn_decode_combine", "attn_fwd_noalloc", "attn_last_device_error", "attn_status_str",
            "attn_version", "attn_set_wait_timeout_ns", "attn_cache_append",
-           "attn_gather_rows")
+           "attn_gather_rows", "attn_topk_fwd")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES in the header
 
 _lib = None
@@ -79,6 +79,9 @@ def load(path: str | None = None):
     lib.attn_gather_rows.restype = i32
     lib.attn_gather_rows.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, Strides,
                                      Strides, i64, vp]
+    lib.attn_topk_fwd.restype = i32
+    lib.attn_topk_fwd.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, vp, vp, i32, i32, i32, i32,
+                                  ctypes.c_float, i32, Strides, Strides, Strides, vp, sz, vp]
     lib.attn_set_wait_timeout_ns.restype = ctypes.c_uint64
     lib.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.attn_last_device_error.restype = i32
@@ -146,6 +149,12 @@ def fwd_raw(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v, scale
     return fn(q, k, v, out, lse, B, Hq, Hkv, Sq, skv_ptr, max_skv, d_k, d_v, float(scale),
               int(causal), dtype_code_, sq, sk, sv, so, workspace_ptr, workspace_nbytes,
               stream_ptr)
+
+
+def topk_raw(*args) -> int:
+    """attn_topk_fwd with raw pointers (ints), in the header's argument
+    order; returns the status code."""
+    return load().attn_topk_fwd(*args)
 
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
@@ -259,6 +268,34 @@ def gather_rows(src: torch.Tensor, dst: torch.Tensor, idx: torch.Tensor, n_sel: 
         raise AttnError(rc, "attn_gather_rows")
 
 
+def topk_fwd(q: torch.Tensor, cache: torch.Tensor, out: torch.Tensor, idx: torch.Tensor,
+             n_sel: torch.Tensor, skv: torch.Tensor, scale: float, lse: torch.Tensor | None,
+             workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+    """attn_topk_fwd: absorbed-MLA decode over the cache rows at idx[b, t],
+    t < n_sel[b], gathered inside the kernel.  q [B, Hq, 1, 576], cache
+    [B, 1, S, 576], out [B, Hq, 1, 512] (views allowed, last dim contiguous);
+    idx int32 [B, >= topk] with topk = idx.shape[1]; n_sel, skv int32 [B]."""
+    B, Hq, _, d_k = q.shape
+    topk = idx.shape[1]
+    for t in (idx, n_sel, skv):
+        if t.dtype != torch.int32:
+            raise TypeError("idx, n_sel and skv must be int32")
+    if idx.dim() != 2 or idx.stride(1) != 1 or not n_sel.is_contiguous() or not skv.is_contiguous():
+        raise ValueError("idx rows and n_sel/skv must be contiguous")
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise TypeError("lse must be a contiguous float32 tensor")
+    _on_one_gpu(q, cache, out, idx, n_sel, skv, lse, workspace)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = load().attn_topk_fwd(q.data_ptr(), cache.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else None, B, Hq, idx.data_ptr(),
+                              idx.stride(0), n_sel.data_ptr(), skv.data_ptr(), topk,
+                              cache.shape[2], d_k, out.shape[-1], float(scale),
+                              dtype_code(q.dtype), _strides4(q), _strides4(cache), _strides4(out),
+                              workspace.data_ptr(), workspace.numel(), st.cuda_stream)
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_topk_fwd")
+
+
 def set_wait_timeout_ns(ns: int) -> int:
     """Bound every device-side wait of later launches (0 = default 2 s);
     returns the previous bound.  Diagnostic only (see the header)."""
@@ -280,12 +317,14 @@ def attention(q, k, v, skv, max_skv, scale, causal=True, with_lse=True, workspac
 
 
 def topk_attention(q, k_cache, v_cache, idx, n_sel, skv, scale, d_v=None, with_lse=True,
-                   scratch=None, stream=None):
-    """Sparse (top-k) decode: attn_gather_rows copies the selected rows of the
-    caches into scratch caches of topk = idx.shape[1] rows, then attn_fwd
-    attends over them, both on one stream.  k_cache/v_cache [B, Hkv, S, d];
-    for an absorbed-MLA latent cache pass v_cache=None and d_v (the value
-    rows are the first d_v columns of the gathered rows).  ``scratch`` is an
+                   scratch=None, stream=None, fused=True):
+    """Sparse (top-k) decode over topk = idx.shape[1] selections per sequence.
+    k_cache/v_cache [B, Hkv, S, d]; for an absorbed-MLA latent cache pass
+    v_cache=None and d_v (the value rows are the first d_v columns of the
+    selected rows).  An absorbed-MLA decode (latent d 576 / 512, one query)
+    runs in one pass, attn_topk_fwd, unless ``fused`` is False; otherwise
+    attn_gather_rows copies the selected rows into scratch caches and
+    attn_fwd attends over them, both on one stream.  ``scratch`` is an
     optional dict the scratch tensors (keys k, v, len, ws) are kept in
     between calls; they are reallocated when the problem's shapes change.
     Returns (out, lse)."""
@@ -296,6 +335,18 @@ def topk_attention(q, k_cache, v_cache, idx, n_sel, skv, scale, d_v=None, with_l
         raise ValueError("d_v is required for a latent (MLA) cache")
     d_v = d_v if latent else v_cache.shape[-1]
     sc = scratch if scratch is not None else {}
+    if fused and latent and d_k == 576 and d_v == 512 and Hkv == 1 and q.shape[2] == 1:
+        key = ("fused", B, topk, q.shape[1], k_cache.device)
+        if sc.get("key") != key:
+            sc.clear()
+            sc["key"] = key
+            n = workspace_bytes(B, q.shape[1], 1, 1, topk, d_k, d_v)
+            sc["ws"] = torch.empty(max(n, 16), dtype=torch.uint8, device=k_cache.device)
+        out = torch.empty(B, q.shape[1], 1, d_v, dtype=q.dtype, device=q.device)
+        lse = (torch.empty(B, q.shape[1], 1, dtype=torch.float32, device=q.device)
+               if with_lse else None)
+        topk_fwd(q, k_cache, out, idx, n_sel, skv, scale, lse, sc["ws"], stream)
+        return out, lse
     key = (B, Hkv, topk, d_k, d_v, latent, k_cache.dtype, k_cache.device, q.shape[1], q.shape[2])
     if sc.get("key") != key:  # (re)allocate for this problem's shapes
         sc.clear()

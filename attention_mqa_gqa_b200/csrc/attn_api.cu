@@ -322,21 +322,22 @@ attn_status_t launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const 
   return ATTN_OK;
 }
 
-template <bool BF16>
+template <bool BF16, bool GATHER = false>
 attn_status_t launch_mla_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const attn::DecodeParams& dp, const attn::CombineParams& cp,
                               const attn_plan_t& pl, cudaStream_t st, int phases, int n_counters) {
   using Tr = attn::MlaPairTraits;
+  constexpr int threads = GATHER ? Tr::THREADS_GATHER : Tr::THREADS;
   if (phases & PHASE_PARTIAL) {
     const bool fused = phases == PHASE_ALL;  // merge in the kernel
     if (fused && launch_prepare<BF16>(dp, n_counters, Tr::DV, st) != ATTN_OK) return ATTN_ECUDA;
     attn::DecodeParams dpp = dp;
     if (!fused) dpp.counters = nullptr;
-    auto kern = attn::mla_pair_kernel<BF16>;
+    auto kern = attn::mla_pair_kernel<BF16, GATHER>;
     set_smem(kern, Tr::SMEM_BYTES);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)pl.grid_ctas, 1, 1);
-    cfg.blockDim = dim3(Tr::THREADS, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -368,6 +369,55 @@ attn_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const
   kern<<<(unsigned)pl.grid_ctas, Tr::THREADS, Tr::SMEM_BYTES, st>>>(mq, mk, mv, pp);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ECUDA;
   return ATTN_OK;
+}
+
+// Decode-path parameters of one problem: the workspace carved into partial
+// outputs, partial LSEs and merge counters (attn_plan's layout).
+void decode_params(const attn_plan_t& pl, int B, int Hq, int Hkv, int Sq, const int32_t* skv, int d_k,
+                   int d_v, float scale_log2, int causal, attn_strides_t so, void* out, float* lse,
+                   void* workspace, attn::DecodeParams* dp, attn::CombineParams* cp) {
+  const int G = Hq / Hkv;
+  const size_t n = (size_t)pl.partials * G * Sq;
+  *dp = attn::DecodeParams{};
+  dp->skv = skv;
+  dp->ws_o = reinterpret_cast<float*>(workspace);
+  dp->ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                        align256(n * d_v * sizeof(float)));
+  dp->B = B;
+  dp->Hq = Hq;
+  dp->Hkv = Hkv;
+  dp->G = G;
+  dp->Sq = Sq;
+  dp->causal = causal;
+  dp->ranges = pl.kv_ranges;
+  dp->head_blocks = pl.head_blocks;
+  dp->scale_log2 = scale_log2;
+  dp->timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);
+  dp->counters = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(workspace) +
+                                                 align256(n * d_v * sizeof(float)) +
+                                                 align256(n * sizeof(float)));
+  dp->out = out;
+  dp->o_sb = so.b;
+  dp->o_sh = so.h;
+  dp->o_ss = so.s;
+  dp->lse = lse;
+  *cp = attn::CombineParams{};
+  cp->ws_o = dp->ws_o;
+  cp->ws_lse = dp->ws_lse;
+  cp->skv = skv;
+  cp->out = out;
+  cp->o_sb = so.b;
+  cp->o_sh = so.h;
+  cp->o_ss = so.s;
+  cp->lse = lse;
+  cp->B = B;
+  cp->Hq = Hq;
+  cp->Hkv = Hkv;
+  cp->G = G;
+  cp->Sq = Sq;
+  cp->DV = d_v;
+  cp->ranges = pl.kv_ranges;
+  cp->tile_shift = decode_pairs(d_k) ? attn::MlaPairTraits::TILE_SHIFT : 7;
 }
 
 template <bool BF16>
@@ -458,47 +508,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
       return ATTN_ECUDA;
     }
     attn::DecodeParams dp{};
-    dp.skv = skv_per_seq;
-    const size_t n = (size_t)pl.partials * G * Sq;
-    dp.ws_o = reinterpret_cast<float*>(workspace);
-    dp.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
-                                         align256(n * d_v * sizeof(float)));
-    dp.B = B;
-    dp.Hq = Hq;
-    dp.Hkv = Hkv;
-    dp.G = G;
-    dp.Sq = Sq;
-    dp.causal = causal;
-    dp.ranges = pl.kv_ranges;
-    dp.head_blocks = pl.head_blocks;
-    dp.scale_log2 = scale_log2;
-    dp.timeout_ns = g_wait_timeout_ns.load(std::memory_order_relaxed);
-    const int n_counters = (int)merge_counters(B, Hkv, pl.head_blocks, d_k);
-    dp.counters = reinterpret_cast<unsigned int*>(
-        reinterpret_cast<uint8_t*>(workspace) + align256(n * d_v * sizeof(float)) +
-        align256(n * sizeof(float)));
-    dp.out = out;
-    dp.o_sb = so.b;
-    dp.o_sh = so.h;
-    dp.o_ss = so.s;
-    dp.lse = lse;
     attn::CombineParams cp{};
-    cp.ws_o = dp.ws_o;
-    cp.ws_lse = dp.ws_lse;
-    cp.skv = skv_per_seq;
-    cp.out = out;
-    cp.o_sb = so.b;
-    cp.o_sh = so.h;
-    cp.o_ss = so.s;
-    cp.lse = lse;
-    cp.B = B;
-    cp.Hq = Hq;
-    cp.Hkv = Hkv;
-    cp.G = G;
-    cp.Sq = Sq;
-    cp.DV = d_v;
-    cp.ranges = pl.kv_ranges;
-    cp.tile_shift = decode_pairs(d_k) ? attn::MlaPairTraits::TILE_SHIFT : 7;
+    decode_params(pl, B, Hq, Hkv, Sq, skv_per_seq, d_k, d_v, scale_log2, causal, so, out, lse,
+                  workspace, &dp, &cp);
+    const int n_counters = (int)merge_counters(B, Hkv, pl.head_blocks, d_k);
     if (d_k == 128)
       return bf16 ? launch_decode<128, 128, 16, true>(mq, mk, mv, dp, cp, pl, st, phases, n_counters)
                   : launch_decode<128, 128, 16, false>(mq, mk, mv, dp, cp, pl, st, phases, n_counters);
@@ -662,6 +675,53 @@ attn_status_t attn_cache_append(void* k_cache, void* v_cache, const void* k_new,
   ap.vn_sh = svn.h;
   attn::cache_append_kernel<<<B, 256, 0, reinterpret_cast<cudaStream_t>(cuda_stream)>>>(ap);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+attn_status_t attn_topk_fwd(const void* q, const void* cache, void* out, float* lse, int B, int Hq,
+                            const int32_t* idx, int64_t idx_stride, const int32_t* n_sel,
+                            const int32_t* skv_per_seq, int topk, int max_skv, int d_k, int d_v,
+                            float scale, attn_dtype_t dtype, attn_strides_t sq, attn_strides_t sc,
+                            attn_strides_t so, void* workspace, size_t workspace_bytes,
+                            void* cuda_stream) {
+  // ---- validation (nothing touches the GPU before this passes)
+  if (!q || !cache || !out || !idx || !n_sel || !skv_per_seq) return ATTN_EINVAL;
+  if (d_k != 576 || d_v != 512) return ATTN_EUNSUPPORTED;  // the absorbed-MLA latent cache
+  if (B <= 0 || Hq <= 0 || topk <= 0 || max_skv <= 0 || idx_stride < topk) return ATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(out)) return ATTN_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_EINVAL;
+  for (const void* ptr : {static_cast<const void*>(idx), static_cast<const void*>(n_sel),
+                          static_cast<const void*>(skv_per_seq)})
+    if (reinterpret_cast<uintptr_t>(ptr) & 3u) return ATTN_EINVAL;
+  if (!strides_ok(sq) || !strides_ok(sc) || !strides_ok(so) || sc.s == 0) return ATTN_EINVAL;
+  if ((Hq > 1 && sq.h == 0) || (B > 1 && (sq.b == 0 || sc.b == 0))) return ATTN_EINVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_EINVAL;
+  attn_plan_t pl;
+  attn_status_t rc = plan_impl(B, Hq, 1, 1, topk, d_k, d_v, dtype, 0, &pl);
+  if (rc != ATTN_OK) return rc;
+  if (pl.workspace_bytes > 0) {
+    if (!workspace || !aligned16(workspace)) return ATTN_EWORKSPACE;
+    if (workspace_bytes < pl.workspace_bytes) return ATTN_EWORKSPACE;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(cuda_stream);
+  CUtensorMap mq, mk, mv;  // K and V come by the kernel's own gathers; the maps stay unused
+  if (!make_q_rows_map(&mq, q, dtype, d_k, Hq, B, sq.h, sq.b, attn::MlaPairTraits::NHC))
+    return ATTN_ECUDA;
+  if (!make_chunk_map(&mk, cache, dtype, d_k, max_skv, 1, B, sc.s, sc.h, sc.b, 2)) return ATTN_ECUDA;
+  if (!make_chunk_map(&mv, cache, dtype, d_v, max_skv, 1, B, sc.s, sc.h, sc.b, 2)) return ATTN_ECUDA;
+  attn::DecodeParams dp{};
+  attn::CombineParams cp{};
+  decode_params(pl, B, Hq, 1, 1, n_sel, d_k, d_v, scale * 1.4426950408889634f, 0, so, out, lse,
+                workspace, &dp, &cp);
+  dp.idx = idx;
+  dp.idx_sb = idx_stride;
+  dp.src = reinterpret_cast<const uint8_t*>(cache);
+  dp.src_sb = sc.b;
+  dp.src_ss = sc.s;
+  dp.src_len = skv_per_seq;
+  const int n_counters = (int)merge_counters(B, 1, pl.head_blocks, d_k);
+  return dtype == ATTN_BF16
+             ? launch_mla_pair<true, true>(mq, mk, mv, dp, cp, pl, st, PHASE_ALL, n_counters)
+             : launch_mla_pair<false, true>(mq, mk, mv, dp, cp, pl, st, PHASE_ALL, n_counters);
 }
 
 attn_status_t attn_gather_rows(const void* src, void* dst, const int32_t* idx,

@@ -63,6 +63,15 @@ struct DecodeParams {
   void* out;                  // [B, Hq, Sq, d_v]
   int64_t o_sb, o_sh, o_ss;   // element strides of out
   float* lse;                 // [B, Hq, Sq] or NULL
+  // Top-k MLA decode with the rows gathered inside the kernel: key j of
+  // sequence b is row idx[b * idx_sb + j] of the latent cache `src` (one
+  // kv head), j < skv[b]; a position outside [0, src_len[b]) reads as a
+  // zero row and sets bit 2 of the device error word.
+  const int32_t* idx;
+  int64_t idx_sb;
+  const uint8_t* src;         // byte address of the cache
+  int64_t src_sb, src_ss;     // element strides of the cache (sequence, row)
+  const int32_t* src_len;     // [B] valid cache rows per sequence
 };
 
 constexpr uint32_t ceil_pow2_cols(uint32_t n) {

@@ -84,6 +84,12 @@ struct MlaPairTraits {
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
   static constexpr int SOFTMAX_THREADS = 256;
   static constexpr int THREADS = 64 + SOFTMAX_THREADS;
+  // Top-k mode (rows gathered in the kernel): warps 10-11 copy the selected
+  // rows; in CTA 1 warp 10 also forwards their arrival to CTA 0 (12 warps
+  // keep the softmax warps' register budget of the dense kernel).
+  static constexpr int GATHER_WARP0 = THREADS / 32;   // 10
+  static constexpr int GATHER_THREADS = 64;
+  static constexpr int THREADS_GATHER = THREADS + GATHER_THREADS;
   static constexpr int TMEM_S = 0;    // S^T double buffer: 2 x 128 columns
   static constexpr int TMEM_O = 256;  // O^T blocks m = 0, 1: 128 columns each
   static_assert(OFF_QT % 1024 == 0 && OFF_PT % 1024 == 0, "operand alignment");
@@ -108,8 +114,8 @@ __device__ __forceinline__ void transposed_warp_sum(float (&v)[NV], int lane) {
   }
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
+template <bool BF16, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? MlaPairTraits::THREADS_GATHER : MlaPairTraits::THREADS, 1)
     mla_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using T = MlaPairTraits;
@@ -166,7 +172,9 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int g = 0; g < T::RING_G; ++g) {
-      mbar_init(full_bar(g), 1);
+      // top-k mode: one arrival per copying thread (when its copies have
+      // landed), plus CTA 1's forwarded arrival on CTA 0's barrier
+      mbar_init(full_bar(g), GATHER ? T::GATHER_THREADS + (cr == 0 ? 1 : 0) : 1);
       mbar_init(empty_bar(g), 1);
     }
     mbar_init(q_full, 1);
@@ -221,7 +229,114 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
   };
 
   if (count > 0) {
-    if (warp == 0 && lane == 0) {
+    if (GATHER && warp >= T::GATHER_WARP0) {
+      // ------------------------------------------------ producer: gathered K/V groups
+      // The same groups in the same order as the copy producer below, each
+      // filled from the selected cache rows with 16-byte cp.async copies,
+      // eight lanes per 128-byte row chunk (coalesced), into the
+      // 128-byte-swizzled layout a TMA copy would produce.  Warp gw copies
+      // rows 64 gw .. 64 gw + 63 of every group; each lane's copies of a group
+      // complete one arrival on the group's barrier.  A tile's row positions
+      // are read once, while the previous tile's groups are copied (within
+      // a piece), and kept for its V groups.  In CTA 1 warp 10 also forwards each group's arrival to CTA 0
+      // two groups later (CTA 0's pair MMAs read this CTA's half of the group;
+      // a proxy fence first: the copies are generic-proxy writes, the MMA
+      // reads through the async proxy).
+      const int gw = warp - T::GATHER_WARP0;
+      const int rsub = lane >> 3, unit = lane & 7;
+      const bool fwd = cr == 1 && gw == 0;
+      const uint32_t lead = mapa_shared(full_bar(0), 0);
+      int grp = 0, fgrp = 0, pending = 0;
+      uint32_t ph = 0, fph = 0;
+      bool ok = true;
+      auto forward_one = [&]() {
+        if (!ok) return;
+        ok = mbar_wait_warp(full_bar(fgrp), fph, abort_flag, p.timeout_ns, 64);
+        if (!ok) return;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (elect_one()) mbar_arrive_remote_cta(lead + 8 * fgrp);
+        __syncwarp();
+        if (++fgrp == T::RING_G) { fgrp = 0; fph ^= 1u; }
+        --pending;
+      };
+      // positions of keys row0 + 128 h + 64 gw + 32 k + lane (-1: a zero row)
+      auto load_pos = [&](int row0, int b, int (&pr)[2][2]) {
+        const int nsel = p.skv[b];
+        const int len = p.src_len[b];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int key = row0 + 128 * h + 64 * gw + 32 * k + lane;
+            int q = -1;
+            if (key >= 0 && key < nsel) {
+              q = p.idx[(int64_t)b * p.idx_sb + key];
+              if (q < 0 || q >= len) {
+                atomicOr(&g_attn_error, 4u);
+                q = -1;
+              }
+            }
+            pr[h][k] = q;
+          }
+      };
+      auto gather = [&](int c0, int nch, const int (&pr)[2], int b) {
+        if (!ok) return;
+        ok = mbar_wait_warp_cluster(empty_bar(grp), ph ^ 1u, abort_flag, p.timeout_ns, 63);
+        if (!ok) return;
+        const uint8_t* sb0 = p.src + (int64_t)b * p.src_sb * 2;
+        const uint32_t gbase = ring + grp * T::GBYTES;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int rl = 4 * i + rsub;  // row within this warp's 64
+          const int q = __shfl_sync(0xffffffffu, pr[rl >> 5], rl & 31);
+          const int r = 64 * gw + rl;   // row within the group
+          const uint8_t* srow = sb0 + (int64_t)(q < 0 ? 0 : q) * p.src_ss * 2 + unit * 16;
+          for (int cc = 0; cc < nch; ++cc)
+            cp_async16(gbase + cc * T::SLOT + r * 128 + ((unit ^ (r & 7)) << 4),
+                       srow + (c0 + cc) * 128, q < 0 ? 0u : 16u);
+        }
+        cp_async_arrive_noinc(full_bar(grp));
+        if (++grp == T::RING_G) { grp = 0; ph ^= 1u; }
+        if (fwd && ++pending > 2) forward_one();
+      };
+      PieceWalker w = walker();
+      int b, kvh, t0, n;
+      int cur[2][2], nxt[2][2], prev[2][2], prev_b = 0;
+      bool have_prev = false;
+      auto gather_v = [&]() {
+        for (int m = 0; m < 2; ++m)
+          for (int h = 0; h < 2; ++h) gather(4 * m + 2 * (int)cr, 2, prev[h], prev_b);
+      };
+      while (ok && w.next(b, kvh, t0, n)) {
+        // a partial last pair tile is the 256 selections ending at the last
+        // one (earlier keys masked); keys before the first are zero rows
+        const int last_win = p.skv[b] - 256;
+        load_pos(min(t0 * 256, last_win), b, nxt);
+        for (int i = 0; i < n && ok; ++i) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            cur[h][0] = nxt[h][0];
+            cur[h][1] = nxt[h][1];
+          }
+          // the next tile's positions load while this tile's groups are copied
+          if (i + 1 < n) load_pos(min((t0 + i + 1) * 256, last_win), b, nxt);
+          if (i == 0 && have_prev) gather_v();
+          for (int c = 0; c < T::KCH; c += 2) gather(c, min(2, T::KCH - c), cur[cr], b);
+          if (i > 0) gather_v();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            prev[h][0] = cur[h][0];
+            prev[h][1] = cur[h][1];
+          }
+          prev_b = b;
+          have_prev = true;
+        }
+      }
+      if (have_prev) gather_v();
+      while (ok && fwd && pending > 0) forward_one();
+      if (!ok) *abort_flag = 1;
+    } else if (!GATHER && warp == 0 && lane == 0) {
       // ------------------------------------------------ producer: K/V groups
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -312,6 +427,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
             ok = mbar_wait_warp_cluster(full_bar(grp), ph, abort_flag, p.timeout_ns, 44);
             if (!ok) return;
             tc_fence_after();
+            if constexpr (GATHER) fence_proxy_async_smem();  // this CTA's cp.async rows
             if (elect_one()) {
               // A = V^T (MN-major, 128-byte swizzle): the group's two chunks are
               // the block's two 64-row halves (LBO = one chunk), 8-key groups
@@ -358,6 +474,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
             ok = mbar_wait_warp_cluster(full_bar(grp), ph, abort_flag, p.timeout_ns, 47);
             if (!ok) break;
             tc_fence_after();
+            if constexpr (GATHER) fence_proxy_async_smem();  // this CTA's cp.async rows
             if (elect_one()) {
               // A = K rows (each CTA its own 128 keys), B = Q^T chunks (each CTA
               // its 64 heads): K-major, 128-byte swizzle, 32 bytes per K step.
@@ -411,7 +528,7 @@ __global__ void __launch_bounds__(MlaPairTraits::THREADS, 1)
           __syncwarp();
         }
       }
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < T::GATHER_WARP0) {
       // ------------------------------------------------ softmax + epilogues
       constexpr int HH = NHC;                  // heads per thread (64)
       const int st = threadIdx.x - 64;         // 0..255

@@ -547,6 +547,19 @@ __device__ __forceinline__ void st_async_f32(uint32_t raddr, float v, uint32_t r
                : "memory");
 }
 
+// 16-byte copy global -> shared by the executing thread (L1 bypassed);
+// `src_bytes` = 0 fills the 16 bytes with zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// Arrive on a local mbarrier once all of this thread's earlier cp.async
+// copies have landed; the arrival is one of the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
 // from this CTA's shared memory to a peer CTA's (`dst` and `rbar` from
 // mapa); the bytes are counted on the peer's mbarrier `rbar`.  The source

@@ -21,8 +21,9 @@ Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and a device synchronize on both sides, replayed from CUDA graphs of two
 steps that hold the steps' C-ABI launches; CUDA events on the replay stream
 (one between consecutive replays for the step-time percentiles).  The dominant kernel's
-duration (and the row gather's, for a top-k step) is timed the same way on
-graphs of 20 back-to-back launches of that kernel alone.  With N GPUs
+duration is timed the same way on graphs of 20 back-to-back launches of that
+kernel alone (a top-k step is one attn_topk_fwd: the decode kernel gathers
+the selected rows itself).  With N GPUs
 (torchrun) every rank runs its own replica of the workload and the time is
 the max over ranks.  Inputs are larger than L2 for the decode workloads (the
 KV cache alone is 302 MB vs 126 MB L2).  Other workloads: --workload
@@ -257,16 +258,13 @@ class GpuRunner:
         self.skv = inp["skv"].to(device)
         self.topk = w.topk
         if self.topk:
-            # the step: gather the selected rows of the latent cache into a
-            # dense cache of topk rows, then the split decode over it
+            # the step: attn_topk_fwd, the MLA decode that gathers the
+            # selected rows of the latent cache itself (one pass)
             if not w.mla:
                 raise ValueError("top-k workloads are defined on the MLA latent cache")
-            self.src_k, self.src_skv = self.k, self.skv
+            self.cache_rows = self.max_skv
             self.idx = inp["idx"].to(device)
             self.n_sel = inp["n_sel"].to(device)
-            sel = torch.empty(w.B, 1, self.topk, w.d_k, dtype=w.dtype, device=device)
-            self.k, self.v = sel, sel[..., : w.d_v]
-            self.skv = torch.empty(w.B, dtype=torch.int32, device=device)
             self.max_skv = self.topk
         self.out = torch.empty(w.B, w.Hq, w.Sq, w.d_v, dtype=w.dtype, device=device)
         self.lse = torch.empty(w.B, w.Hq, w.Sq, dtype=torch.float32, device=device)
@@ -277,6 +275,15 @@ class GpuRunner:
         self._args = None
 
     def args(self):
+        if self._args is None and self.topk:
+            b, w = self.b, self.w
+            st = lambda t: b.Strides(t.stride(0), t.stride(1), t.stride(2))
+            self._args = (self.q.data_ptr(), self.k.data_ptr(), self.out.data_ptr(),
+                          self.lse.data_ptr(), w.B, w.Hq, self.idx.data_ptr(), self.idx.stride(0),
+                          self.n_sel.data_ptr(), self.skv.data_ptr(), self.topk, self.cache_rows,
+                          w.d_k, w.d_v, w.scale, b.dtype_code(w.dtype), st(self.q), st(self.k),
+                          st(self.out), self.ws.data_ptr(), self.ws.numel(),
+                          self.stream.cuda_stream)
         if self._args is None:
             b, w = self.b, self.w
             st = lambda t: b.Strides(t.stride(0), t.stride(1), t.stride(2))
@@ -288,17 +295,14 @@ class GpuRunner:
                           self.stream.cuda_stream)
         return self._args
 
-    def gather(self):
-        self.b.gather_rows(self.src_k, self.k, self.idx, self.n_sel, self.src_skv, self.skv,
-                           self.stream)
-
     def call(self, entry="attn_fwd"):
-        """One launch group: "attn_fwd" (a whole step; for top-k, the row
-        gather first), "forward" (attn_fwd without the gather), "gather"."""
-        if entry == "gather":
-            return self.gather()
-        if self.topk and entry == "attn_fwd":
-            self.gather()
+        """One launch group: "attn_fwd" = "forward" (a whole step: attn_fwd,
+        or attn_topk_fwd for a top-k workload)."""
+        if self.topk:
+            rc = self.b.topk_raw(*self.args())
+            if rc != 0:
+                raise self.b.AttnError(rc, "attn_topk_fwd")
+            return
         if entry == "forward":
             entry = "attn_fwd"
         rc = self.b.fwd_raw(*self.args(), entry=entry)
@@ -310,7 +314,7 @@ class GpuRunner:
         return self.plan["path"] == 1
 
     def launches_per_step(self):
-        return (2 if self.decode else 1) + (1 if self.topk else 0)
+        return 2 if self.decode else 1
 
     def _graph(self, nsteps, entry="attn_fwd"):
         """Capture `nsteps` launches of `entry` (a whole step for attn_fwd)
@@ -356,8 +360,7 @@ class GpuRunner:
         20 back-to-back launches of it alone: for decode, attn_fwd's split
         kernel with the merge of the pieces inside it (with the few-
         microsecond kernel that zeroes its arrival counters and lets it start
-        early); for a top-k step the row gather is timed on its own too (in
-        ``self.gather_ms``), the rest of the step being the other time."""
+        early); for a top-k step the same, the kernel gathering the rows."""
         per = steps_per_graph(steps)
         graph, side = self._graph(per)
         reps = []
@@ -369,12 +372,7 @@ class GpuRunner:
         kg, kside = self._graph(20, "forward")
         k_ms = self._replay_ms(kg, kside, 10, 1) / 200
         del kg
-        self.gather_ms = 0.0
-        if self.topk:
-            gg, gside = self._graph(20, "gather")
-            self.gather_ms = self._replay_ms(gg, gside, 10, 1) / 200
-            del gg
-        return total, k_ms, max(total / steps - k_ms - self.gather_ms, 0.0)
+        return total, k_ms, max(total / steps - k_ms, 0.0)
 
     def e2e(self, steps, warmup, inp):
         """Same step through the C ABI with the step's inputs in pinned host
@@ -386,7 +384,7 @@ class GpuRunner:
         hq = pin(inp["q"])
         hskv = pin(inp["skv"])
         hk = hv = hidx = hnsel = None
-        dskv = self.src_skv if self.topk else self.skv
+        dskv = self.skv
         if not self.decode:  # prefill shapes have separate K and V tensors
             hk, hv = pin(inp["k"]), pin(inp["v"])
         if self.topk:
@@ -771,12 +769,8 @@ def main():
     value = work_all * steps / (max_ms * 1e-3) / scale_div
     metric, unit, hib = metric_of(w)
     roof = dominant_roofline(w, g, keys, k_ms, other_ms, total_ms, peaks, peak_src)
-    if w.topk:  # the row gather: reads and writes the selected rows once each
-        gb = 2 * kv_bytes(w, keys) / (g.gather_ms * 1e-3) / 1e9
-        roof["gather"] = {"kernel": "gather_rows_kernel", "ms": round(g.gather_ms, 5),
-                          "bytes_per_launch": 2 * kv_bytes(w, keys), "achieved": round(gb, 1),
-                          "frac": round(gb / float(peaks["hbm_gbs"]), 4), "unit": "GB/s",
-                          "traffic": traffic_for("gather_rows_kernel", w.name)}
+    if w.topk:
+        roof["gather"] = "in kernel (cp.async rows into the decode kernel's ring)"
 
     # end to end through the C ABI with host buffers
     e2e_steps = max(10, min(steps, 200))

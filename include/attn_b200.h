@@ -250,6 +250,32 @@ attn_status_t attn_gather_rows(const void* src, void* dst, const int32_t* idx,
                                attn_strides_t s_src, attn_strides_t s_dst, int64_t idx_stride,
                                void* cuda_stream);
 
+/*
+ * Top-k sparse absorbed-MLA decode in one pass (the same passage: attention
+ * over the cached entries an indexer selected): out[b, h] = attention of
+ * q[b, h] over the rows at positions idx[b * idx_stride + t], t < n_sel[b],
+ * of the latent cache [B, 1, >= skv[b], 576] (k = whole rows, v = their first
+ * 512 columns), equal to attn_gather_rows followed by attn_fwd, but the rows
+ * are copied straight from the cache into the decode kernel's shared memory,
+ * so each selected byte crosses HBM once.
+ * - q [B, Hq, 1, 576], out [B, Hq, 1, 512], lse [B, Hq, 1] or NULL; element
+ *   strides sq / sc (cache) / so, innermost contiguous, 16-byte aligned.
+ * - idx, n_sel, skv_per_seq: device int32; 0 <= n_sel[b] <= topk (not
+ *   checked on the device); idx_stride >= topk.  A position outside
+ *   [0, skv_per_seq[b]) reads as a zero row and sets bit 2 of the device
+ *   error word (ATTN_EINDEX from attn_last_device_error).
+ * - max_skv: row extent of the cache; workspace: attn_workspace_bytes(B, Hq,
+ *   1, 1, topk, 576, 512) bytes, 16-byte aligned, owned by the caller.
+ * - Errors before launch: ATTN_EINVAL, ATTN_EUNSUPPORTED (d_k != 576 or
+ *   d_v != 512, or what attn_plan refuses), ATTN_EWORKSPACE, ATTN_ECUDA.
+ */
+attn_status_t attn_topk_fwd(const void* q, const void* cache, void* out, float* lse, int B, int Hq,
+                            const int32_t* idx, int64_t idx_stride, const int32_t* n_sel,
+                            const int32_t* skv_per_seq, int topk, int max_skv, int d_k, int d_v,
+                            float scale, attn_dtype_t dtype, attn_strides_t sq, attn_strides_t sc,
+                            attn_strides_t so, void* workspace, size_t workspace_bytes,
+                            void* cuda_stream);
+
 /* Bound on every device-side wait of launches made after this call, in
  * nanoseconds of %globaltimer (process-wide; 0 restores the default of 2 s).
  * Returns the previous bound.  A diagnostic: a bound far below a kernel's

@@ -1,9 +1,11 @@
 """Top-k sparse decode (DSA style, "带你了解Attention" section 5.1): the rows
 at caller-selected positions are gathered (attn_gather_rows) and attention
-runs over them (attn_fwd); compared with the oracle's attention over the
-selected subset.  Also: the gathered rows are bitwise copies, ragged and
-empty selections, a position outside its sequence reported as ATTN_EINDEX,
-and every output of the full-size 2048-of-16K..48K MLA workload."""
+runs over them (attn_fwd), or, for absorbed MLA, the decode kernel gathers
+them itself (attn_topk_fwd); both compared with the oracle's attention over
+the selected subset, and with each other bitwise.  Also: the gathered rows
+are bitwise copies, ragged and empty selections, a position outside its
+sequence reported as ATTN_EINDEX by both paths, and every output of the
+full-size 2048-of-16K..48K MLA workload."""
 import math
 
 import pytest
@@ -47,9 +49,15 @@ def _run(name, skv, topk, seed, n_sel_override=None):
     sc = {}
     out, lse = binding.topk_attention(dev["q"], dev["k"], None if c["mla"] else dev["v"],
                                       idx.cuda(), n_sel.cuda(), dev["skv"], w.scale,
-                                      d_v=c["dv"], scratch=sc)
+                                      d_v=c["dv"], scratch=sc, fused=False)
     torch.cuda.synchronize()
     assert binding.last_device_error() == binding.ATTN_OK
+    if c["mla"]:  # the one-pass path: the same kernel on the same rows, bit for bit
+        out_f, lse_f = binding.topk_attention(dev["q"], dev["k"], None, idx.cuda(), n_sel.cuda(),
+                                              dev["skv"], w.scale, d_v=c["dv"])
+        torch.cuda.synchronize()
+        assert binding.last_device_error() == binding.ATTN_OK
+        assert torch.equal(out_f, out) and torch.equal(lse_f, lse)
     # the gathered rows are bitwise copies of the selected cache rows
     kg = sc["k"].cpu()
     assert torch.equal(sc["len"].cpu(), n_sel)
@@ -96,6 +104,28 @@ def test_topk_position_outside_sequence_reports_eindex():
     assert torch.equal(dst[1, 0, 2], src[1, 0, 3])
     assert (dst[:, :, 4:].float() == 7.0).all() and (dst[1, :, 3:].float() == 7.0).all()
     assert dlen.tolist() == [4, 3]
+
+
+def test_topk_fused_position_outside_sequence_reports_eindex():
+    """attn_topk_fwd reads a position outside its sequence as a zero row (as
+    the gather pass writes it) and reports ATTN_EINDEX."""
+    from attention_mqa_gqa_b200 import binding
+
+    B, Hq, S = 2, 128, 300
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(B, Hq, 1, 576, generator=g).to(torch.bfloat16).cuda()
+    cache = torch.randn(B, 1, S, 576, generator=g).to(torch.bfloat16).cuda()
+    idx = torch.tensor([[0, 5, 299, 2, 7, 9], [1, 300, 3, -1, 0, 0]], dtype=torch.int32,
+                       device="cuda")
+    n_sel = torch.tensor([4, 4], dtype=torch.int32, device="cuda")
+    skv = torch.tensor([S, S], dtype=torch.int32, device="cuda")
+    ref, ref_lse = binding.topk_attention(q, cache, None, idx, n_sel, skv, 0.07, d_v=512,
+                                          fused=False)
+    assert binding.last_device_error() == binding.ATTN_EINDEX
+    out, lse = binding.topk_attention(q, cache, None, idx, n_sel, skv, 0.07, d_v=512)
+    assert binding.last_device_error() == binding.ATTN_EINDEX
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
 
 
 def test_full_workload():
