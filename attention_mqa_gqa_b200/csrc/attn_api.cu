@@ -236,8 +236,20 @@ enum : int { PHASE_PARTIAL = 1, PHASE_COMBINE = 2, PHASE_ALL = 3 };
 template <bool BF16>
 attn_status_t launch_prepare(const attn::DecodeParams& dp, int n_counters, int d_v,
                              cudaStream_t st) {
-  attn::decode_prepare_kernel<BF16><<<4, 256, 0, st>>>(dp, n_counters, d_v);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(4, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn::decode_prepare_kernel<BF16>, dp, n_counters, d_v) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ECUDA;
+  }
+  return ATTN_OK;
 }
 
 // The combine is launched with programmatic stream serialization: its blocks

@@ -406,12 +406,16 @@ __device__ __forceinline__ int unit_pieces(long long gstart, int tile0, int tb, 
 
 // Zeroes the arrival counters of the in-kernel merge and writes the output
 // of sequences with no key (out = 0, LSE = -inf): no piece covers them.
-// Lets the decode kernel, launched after it with programmatic stream
-// serialization, start at once; that kernel waits for this one to finish
-// only before its first counter update.
+// Launched with programmatic stream serialization, so that it is resident
+// before the previous kernel of the stream ends; it waits for that kernel
+// (and all earlier work) to complete, then lets the decode kernel, launched
+// after it the same way, start at once -- that kernel reads its inputs
+// right away and waits for this one to finish only before its first counter
+// update.
 template <bool BF16>
 __global__ void __launch_bounds__(256) decode_prepare_kernel(const DecodeParams p, int n_counters,
                                                              int DV) {
+  pdl_wait();
   pdl_launch_dependents();
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nth = gridDim.x * blockDim.x;
