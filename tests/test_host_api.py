@@ -208,6 +208,37 @@ def test_fwd_rejects_before_launch(lib, over, code):
 
 
 @pytest.mark.parametrize("over,code", [
+    (dict(q=None), binding.ATTN_EINVAL),
+    (dict(idx=None), binding.ATTN_EINVAL),
+    (dict(n_sel=None), binding.ATTN_EINVAL),
+    (dict(n_sel=0x50002), binding.ATTN_EINVAL),          # int32 array not 4-byte aligned
+    (dict(cache=0x20008), binding.ATTN_EINVAL),          # not 16-byte aligned
+    (dict(idx_stride=100), binding.ATTN_EINVAL),         # rows shorter than topk
+    (dict(topk=0), binding.ATTN_EINVAL),
+    (dict(max_skv=0), binding.ATTN_EINVAL),
+    (dict(sc=binding.Strides(256 * 576, 256 * 576, 0)), binding.ATTN_EINVAL),  # row stride 0
+    (dict(scale=0.0), binding.ATTN_EINVAL),
+    (dict(dtype=7), binding.ATTN_EINVAL),
+    (dict(d_k=512, d_v=512), binding.ATTN_EUNSUPPORTED),  # the one-pass path is MLA only
+    (dict(ws=None), binding.ATTN_EWORKSPACE),
+    (dict(ws_n=64), binding.ATTN_EWORKSPACE),
+])
+def test_topk_fwd_rejects_before_launch(lib, over, code):
+    """attn_topk_fwd validates its arguments before anything reaches the
+    device (the fake pointers below are never dereferenced)."""
+    a = dict(q=0x10000, cache=0x20000, out=0x40000, lse=None, B=2, Hq=128, idx=0x70000,
+             idx_stride=256, n_sel=0x50000, skv=0x58000, topk=256, max_skv=4096, d_k=576,
+             d_v=512, scale=0.07, dtype=0, sq=binding.Strides(128 * 576, 576, 576),
+             sc=binding.Strides(4096 * 576, 4096 * 576, 576),
+             so=binding.Strides(128 * 512, 512, 512), ws=0x60000, ws_n=1 << 30)
+    a.update(over)
+    assert binding.topk_raw(a["q"], a["cache"], a["out"], a["lse"], a["B"], a["Hq"], a["idx"],
+                            a["idx_stride"], a["n_sel"], a["skv"], a["topk"], a["max_skv"],
+                            a["d_k"], a["d_v"], a["scale"], a["dtype"], a["sq"], a["sc"], a["so"],
+                            a["ws"], a["ws_n"], None) == code
+
+
+@pytest.mark.parametrize("over,code", [
     (dict(kc=None), binding.ATTN_EINVAL),
     (dict(skv=None), binding.ATTN_EINVAL),
     (dict(dk=100), binding.ATTN_EINVAL),                 # not a multiple of 8 elements
