@@ -437,8 +437,8 @@ def value_of(w, skv, ms):
 
 
 def roofline(w, skv, kernel_ms, peaks, peak_src, long_run, traffic):
-    """Roofline of the dominant kernel: `frac` against the measured peak of
-    this machine's B200s (MEASURED_PEAKS.json, else the fallback figures), and
+    """Roofline of the dominant kernel: `frac` against the measured B200
+    peaks (MEASURED_PEAKS.json, else the fallback figures), and
     `frac_nominal` against the datasheet figure (~8 TB/s HBM, 2.25 PFLOP/s
     dense bf16), each labelled with its denominator."""
     if w.is_decode:
