@@ -38,6 +38,12 @@
 // each) and the epilogue.  All waits are bounded; the CTAs meet in a
 // hardware cluster barrier only after both have left every loop.
 //
+// Gather mode (top-k decode, 384 threads): the keys of a sequence are the
+// cache rows at caller-selected positions.  Warp 0 lane 0 is idle; warps
+// 10-11 fill the same ring groups in the same order with 16-byte cp.async
+// copies of the selected rows (so each selected byte crosses HBM once),
+// and in CTA 1 warp 10 forwards each group's arrival to CTA 0.
+//
 // Cross-CTA traffic avoids cluster-scope release arrivals, which stall the
 // arriving thread for about a microsecond while the SM streams copies: data
 // (tile maxima, row sums, P^T rows) goes by st.async, whose bytes complete

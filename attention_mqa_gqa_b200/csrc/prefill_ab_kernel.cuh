@@ -9,10 +9,11 @@
 //
 //   CTA 0 ("scores"):  Q (bf16/fp16) in TMEM columns 256..511, copied there
 //       once per item; S[128 x 128 keys] = Q K^T by TMEM-operand UMMAs into
-//       two S buffers (columns 0..255); the online softmax (four threads per
-//       query row) turns each 64-key half of S into P, writes it into a
-//       local staging buffer and ships it to CTA 1's shared memory with
-//       bulk copies (four 4 KB copies per half, one per 32-row quarter).
+//       two S buffers (columns 0..255); the online softmax (one thread per
+//       query row and 64-key half of the tile) turns each half of S into P,
+//       writes it into that half's local staging buffer and ships it to
+//       CTA 1's shared memory with bulk copies (one 4 KB copy per warp: its
+//       32 rows).
 //   CTA 1 ("output"):  O[128 x 512] in all of its TMEM; O += P V over each
 //       64-key half (two UMMAs of N = 256); when a row's running maximum
 //       was raised it rescales O in TMEM first; at the end of the item
@@ -25,20 +26,22 @@
 // ("GQA和MLA详解" section 1: prefill is the quadratic, compute-bound phase;
 // "带你了解Attention" section 6.3: tiling with an online softmax.)
 //
-// Roles (576 threads per CTA):
+// Roles (608 threads per CTA):
 //   CTA 0: warp 0 lane 0 copies Q and K (TMA); warp 1 copies Q into TMEM
-//       and issues the S UMMAs; warps 2-17 run the softmax.
+//       and issues the S UMMAs; warps 2-9 run the softmax (warp w: TMEM lane
+//       quarter w % 4, tile half (w - 2) / 4); warps 10-18 are idle.
 //   CTA 1: warp 0 lane 0 copies V; warp 1 issues the PV UMMAs and posts
 //       events (rescale, end of item) to warps 2-17, which rescale O or
-//       write the output.
+//       write the output; warp 18 watches the P buffers fill and tells CTA
+//       0 when a staged half has landed.
 // Cross-CTA traffic: P by cp.async.bulk from CTA 0's staging buffers (on
 // this part a bulk copy moves shared memory to the peer SM about twice as
-// fast as st.async), rescale factors, partial row sums and row maxima by
-// st.async (all bytes counted on CTA 1 mbarriers); "P buffer free" by
-// tcgen05.commit multicast from CTA 1's MMA issuer; "staging buffer read"
-// and "row sums read" by relaxed remote arrivals from CTA 1.  All waits are
-// bounded; the two CTAs meet in a hardware cluster barrier only after both
-// have left every loop.
+// fast as st.async), rescale factors, the halves' row sums and the row
+// maxima by st.async (all bytes counted on CTA 1 mbarriers); "P buffer
+// free" by tcgen05.commit multicast from CTA 1's MMA issuer; "staging
+// buffer landed" and "row sums read" by relaxed remote arrivals from CTA 1.
+// All waits are bounded; the two CTAs meet in a hardware cluster barrier
+// only after both have left every loop.
 #pragma once
 
 #include "prefill_kernel.cuh"
