@@ -461,27 +461,23 @@ __global__ void __launch_bounds__(PrefillABTraits::THREADS, 1)
         // the previous tile).
         const bool whole = win0 == tile0 && tile0 + T::KT <= lim;
         // pass 1: the row maximum of the raw scores over the tile (scale > 0
-        // keeps the order); the next 32 columns load while these are folded
+        // keeps the order), in two 64-column loads (each wait for TMEM data
+        // costs about as much as folding 64 values)
         float mx = -INFINITY;
-        {
-          float v[2][32];
-          tmem_ld<32>(srow, v[0]);
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[64];
+          tmem_ld<64>(srow + 64 * c, v);
           tmem_wait_ld();
+          if (whole) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c < 3) tmem_ld<32>(srow + 32 * (c + 1), v[(c + 1) & 1]);
-            const float* w = v[c & 1];
-            if (whole) {
+            for (int e = 0; e < 64; e += 2) mx = fmaxf(mx, fmaxf(v[e], v[e + 1]));
+          } else {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) mx = fmaxf(mx, fmaxf(w[e], w[e + 1]));
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int key = win0 + 32 * c + e;
-                if (key >= tile0 && key < lim) mx = fmaxf(mx, w[e]);
-              }
+            for (int e = 0; e < 64; ++e) {
+              const int key = win0 + 64 * c + e;
+              if (key >= tile0 && key < lim) mx = fmaxf(mx, v[e]);
             }
-            if (c < 3) tmem_wait_ld();
           }
         }
         const float tm = mx * p.scale_log2;
