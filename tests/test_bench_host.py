@@ -122,3 +122,28 @@ def test_clock_sampler_summary(tmp_path):
     assert cs.stop() == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
                          "samples": 3}
     assert not os.path.exists(cs.path)
+
+
+def test_dominant_kernel_names():
+    """The roofline names the kernel each path runs (d = 512 prefill: the
+    split-matmul pairs), and every named kernel has its sources listed, so a
+    recorded traffic figure can be matched to the code it was taken on."""
+
+    class G:
+        def __init__(self, decode):
+            self.decode = decode
+
+    names = set()
+    for name, w in wl.WORKLOADS.items():
+        k = bench.kernel_name(w, G(w.is_decode))
+        names.add(k)
+        if not w.is_decode:
+            assert k == ("prefill_ab_kernel" if w.d_k == 512 else "prefill_kernel"), name
+        elif w.mla:
+            assert k == "mla_pair_kernel", name
+        else:
+            assert k == "decode_split_kernel", name
+    assert names <= set(bench.KERNEL_SOURCES)
+    for srcs in bench.KERNEL_SOURCES.values():
+        for f in srcs:
+            assert os.path.exists(os.path.join(bench.ROOT, f)), f
